@@ -1,0 +1,151 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) block-sparse attention library
+ *          (libbsa_b200.so): content-aware block masks (ASA), fixed block
+ *          patterns, and attention over the kept blocks.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors Q, K, V, O are bf16, shape [B, H, N, d], contiguous, row-major
+ *    (d fastest).  LSE is fp32 [B, H, N].  Token order inside N is whatever the
+ *    caller uses (the video layers are frame-major (t, y, x), x fastest).
+ *  - Blocks: nb = ceil(N / blk) query blocks and nb key/value blocks (self
+ *    attention).  Block i holds tokens [i*blk, min((i+1)*blk, N)); the last one
+ *    may be partial.
+ *  - A block mask is CSR over rows r = (b*H + h)*nb + i:
+ *      row_ptr int32 [B*H*nb + 1], row_ptr[0] = 0, non-decreasing;
+ *      col_idx int32 [row_ptr[B*H*nb]], each row's kv-block ids strictly
+ *      ascending, each in [0, nb).
+ *  - Every pointer argument is a DEVICE pointer owned by the caller unless its
+ *    name ends in _host.  The library allocates no device memory: scratch comes
+ *    from a caller-supplied workspace sized by the matching *_workspace_size().
+ *    Workspaces must be 256-byte aligned; Q/K/V/O must be 16-byte aligned.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream) unless
+ *    stated otherwise, and returns a status code.  Arguments are validated on
+ *    the host first: an invalid call returns an error and launches nothing.
+ *    Errors found on the device (capacity overflow, malformed CSR, a bounded
+ *    wait that gave up) are recorded in a per-device status word read by
+ *    bsa_check_device_status().  No C++ exception crosses this interface.
+ *  - Supported: d in {64, 128}; blk in {16, 32, 64, 128}; N >= 1; B, H >= 1;
+ *    B*H*nb*nb < 2^31.  The device must be sm_100 (B200).
+ *
+ * Sources (web pages on the method):
+ *  [BLADE]   "BLADE: Block-Sparse Attention Meets Step Distillation for
+ *            Efficient Video Generation" (digest: abstract; 方法详解 / 关键设计)
+ *  [SvDiT]   "Sparse-vDiT: Sparse Attention Acceleration for Video Diffusion
+ *            Transformers" (blog: 核心公式; 四种注意力模式 table; 模型组件)
+ *  [EvDiT]   "Efficient-vDiT: Efficient Video Diffusion Transformers With
+ *            Attention Tile" (blog: 3.1 注意力图块化)
+ */
+#ifndef BSA_B200_H
+#define BSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* bsa_stream_t; /* same object as cudaStream_t */
+
+/* ---- status codes ------------------------------------------------------- */
+#define BSA_OK               0
+#define BSA_ERR_INVALID_ARG (-1) /* null pointer, non-positive size, bad mode   */
+#define BSA_ERR_UNSUPPORTED (-2) /* d, blk, alignment or size outside support   */
+#define BSA_ERR_CAPACITY    (-3) /* col_idx capacity too small for the mask     */
+#define BSA_ERR_CUDA        (-4) /* a CUDA runtime call or launch failed        */
+#define BSA_ERR_TIMEOUT     (-5) /* a device-side bounded wait gave up          */
+#define BSA_ERR_CSR         (-6) /* device saw a block index outside [0, nb)    */
+#define BSA_ERR_WORKSPACE   (-7) /* workspace null, too small or misaligned     */
+
+#define BSA_MODE_TOPK 0
+#define BSA_MODE_MASS 1
+
+#define BSA_PATTERN_FULL      0 /* M0  [SvDiT] every block                          */
+#define BSA_PATTERN_SKIP      1 /* M1  [SvDiT] head skipped, output zero            */
+#define BSA_PATTERN_DIAG      2 /* M2  [SvDiT] diagonal band (intra-frame)          */
+#define BSA_PATTERN_MULTIDIAG 3 /* M3  [SvDiT] diagonals at frame offsets           */
+#define BSA_PATTERN_STRIPE    4 /* M4  [SvDiT] vertical stripes (global tokens)     */
+#define BSA_PATTERN_TILE3D    5 /*     [EvDiT] frame tiles + global frames          */
+
+/* ---- ASA: content-aware block mask --------------------------------------
+ * [BLADE] ASA generates, per input, a sparsity mask that keeps the block pairs
+ * whose mutual relevance is high.  The pages do not define the score; this
+ * library computes, per (b, h):
+ *   1. pooled q̄_i, k̄_j = mean of the block's valid rows (fp32 accumulation);
+ *   2. s_ij = q̄_i·k̄_j·scale (scale = 1/sqrt(d) when softmax_scale <= 0, the
+ *      attention scale of [SvDiT] 核心公式); p_i = softmax_j s_i over all nb;
+ *   3. order j by (p desc, j asc);
+ *      mode BSA_MODE_TOPK: the first `topk`;
+ *      mode BSA_MODE_MASS: the shortest prefix with cumulative p >= mass_tau;
+ *   4. cap: when max_keep_ratio > 0 keep at most max(1, floor(max_keep_ratio*nb));
+ *   5. union with the diagonal block i (keep_diag != 0) and blocks
+ *      [0, n_sink_blocks);
+ *   6. write CSR (row_ptr, col_idx ascending).
+ * Selection runs in fp32 on the device: rows whose result depends on scores
+ * within fp32 rounding of the cut may differ from an exact evaluation.
+ * q, k: bf16 [B,H,N,d].  col_capacity: entries available in col_idx; if the mask
+ * needs more, entries past the capacity are not written and the device status
+ * becomes BSA_ERR_CAPACITY.  asa_build_mask_max_nnz() gives a bound that never
+ * overflows.  Workspace: asa_build_mask_workspace_size() bytes. */
+size_t  asa_build_mask_workspace_size(int B, int H, int N, int d, int blk);
+int64_t asa_build_mask_max_nnz(int B, int H, int N, int blk, int mode, int topk,
+                               float max_keep_ratio, int keep_diag, int n_sink_blocks);
+int asa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int blk,
+                   int mode, int topk, float mass_tau, float max_keep_ratio,
+                   int keep_diag, int n_sink_blocks, float softmax_scale,
+                   int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                   void* workspace, size_t ws_bytes, bsa_stream_t stream);
+
+/* ---- fixed patterns ------------------------------------------------------
+ * [SvDiT] 四种注意力模式 (M0 full, M1 skip, M2 diagonal, M3 multi-diagonal,
+ * M4 vertical stripe) and [EvDiT] 3.1 (3D attention tile), one pattern per
+ * head, rows replicated over b.  Block (i, j) is kept when some token pair
+ * (t in block i, u in block j, both < N) satisfies the pattern's rule, with
+ * S = frame_tokens:
+ *   FULL      always;            SKIP  never (row empty -> O = 0, LSE = -inf);
+ *   DIAG      |i - j| <= band_w  (block bandwidth);
+ *   MULTIDIAG |u - t - f*S| <= band_w*blk for some f in [f_lo, f_hi];
+ *   STRIPE    (u mod S) < stripe_blocks*blk   (leading tokens of every frame);
+ *   TILE3D    floor(u/S) == floor(t/S) or floor(u/S) < tile_global_frames.
+ * head_pattern_host: HOST int32 [H].  If nnz_out_host is non-NULL the call
+ * synchronizes `stream` once after counting, stores the mask's nnz there, and
+ * returns BSA_ERR_CAPACITY (writing no col_idx) when col_capacity < nnz.  With
+ * nnz_out_host NULL the call is fully asynchronous and an overflow is reported
+ * through the device status.  No workspace. */
+int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
+                 int band_w, int frame_tokens, int f_lo, int f_hi, int stripe_blocks,
+                 int tile_global_frames, int32_t* row_ptr, int32_t* col_idx,
+                 int64_t col_capacity, int64_t* nnz_out_host, bsa_stream_t stream);
+
+/* ---- attention over kept blocks -------------------------------------------
+ * [SvDiT] 核心公式: O = softmax(Q Kᵀ · scale) V per head, here for each query
+ * token t of block i over the key tokens (< N) of the blocks listed in CSR row
+ * (b*H + h)*nb + i only ([BLADE] abstract: computation focused on the kept
+ * blocks).  scale = 1/sqrt(d) when softmax_scale <= 0.
+ * Output: o bf16 [B,H,N,d] (round to nearest even), lse fp32 [B,H,N] =
+ * ln Σ_u exp(q_t·k_u·scale); an empty row gives o = 0 and lse = -inf
+ * ([SvDiT] M1: a skipped head outputs zero).  lse may be NULL.
+ * Accumulation is fp32 on the tensor cores (tcgen05, operands from TMA-loaded
+ * shared memory).  A CSR block id outside [0, nb) is skipped and flagged
+ * (BSA_ERR_CSR in the device status).  Workspace: bsa_forward_workspace_size()
+ * bytes (may be 0, then workspace may be NULL). */
+size_t bsa_forward_workspace_size(int B, int H, int N, int d, int blk);
+int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                int blk, const int32_t* row_ptr, const int32_t* col_idx,
+                float softmax_scale, void* o, float* lse,
+                void* workspace, size_t ws_bytes, bsa_stream_t stream);
+
+/* ---- status ----------------------------------------------------------------
+ * bsa_check_device_status synchronizes `stream`, returns the first error any
+ * kernel of this library recorded on the current device since the last check
+ * (BSA_OK if none), and clears it.  bsa_status_string never returns NULL. */
+int bsa_check_device_status(bsa_stream_t stream);
+const char* bsa_status_string(int status);
+/* Library version as major*10000 + minor*100 + patch. */
+int bsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_B200_H */
