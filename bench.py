@@ -1,0 +1,391 @@
+#!/usr/bin/env python
+"""Benchmark of the block-sparse attention layer (ASA mask + attention over the
+kept blocks) on B200, one process per GPU.
+
+A step is one pass of the hot path over one layer: asa_build_mask (pool, score
+and select, CSR) followed by bsa_forward, through the C ABI.  The default
+workload is the Wan2.1-1.3B-shaped self-attention layer (B1 H12 N32760 d128,
+block 64, cumulative mass 0.9 capped at keep ratio 0.1).  The metric is the
+effective TFLOPS over computed blocks: Σ over kept (q-block, kv-block) pairs of
+4·n_q·n_k·d with valid tokens only, divided by the step time.
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload wan|cog|hunyuan|tiny]
+  python bench.py --impl reference      # the fp64 CPU oracle on a bounded sample
+
+Under torchrun every rank runs its own replica of the layer (the path has no
+cross-GPU exchange); the timed region is bracketed by barriers and the maximum
+over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_attention_asa_b200 import workloads as W  # noqa: E402
+
+METRIC = "block-sparse attn effective TFLOPS & % BF16 TC peak; ms/layer at keep ratio"
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_HBM_GBS = 8000.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+def workload(name: str) -> W.Workload:
+    return {"wan": W.WAN, "cog": W.COG, "hunyuan": W.HUNYUAN, "tiny": W.TINY}[name]
+
+
+def block_flops(w: W.Workload, row_ptr: np.ndarray, col_idx: np.ndarray) -> float:
+    """Σ over kept (row, kv-block) of 4·n_q·n_k·d on valid tokens."""
+    nb = w.nb
+    sizes = np.full(nb, w.blk, dtype=np.float64)
+    sizes[-1] = w.N - (nb - 1) * w.blk
+    rows = len(row_ptr) - 1
+    counts = np.diff(row_ptr.astype(np.int64))
+    i_of_row = np.arange(rows) % nb
+    nq = np.repeat(sizes[i_of_row], counts)
+    nk = sizes[col_idx[:int(row_ptr[-1])]]
+    return float(4.0 * w.d * np.sum(nq * nk))
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup(n_gpus: int):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def barrier_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_inputs(w: W.Workload, heads: int):
+    """fp64 inputs of the first `heads` heads of the layer (drawn like the GPU's)."""
+    q, k, v = W.make_qkv(w)
+    return tuple(W.as_f64(t[:, :heads].contiguous()) for t in (q, k, v))
+
+
+def oracle_step(w: W.Workload, qkv, heads: int):
+    """One oracle pass (ASA mask + masked attention) over the sample: (seconds, flops)."""
+    import oracle
+    qf, kf, vf = qkv
+    t0 = time.perf_counter()
+    m = oracle.asa_mask(qf, kf, w.blk, w.mode, w.topk, w.mass_tau, w.max_keep_ratio, w.keep_diag,
+                        w.n_sink_blocks)
+    oracle.masked_attention(qf, kf, vf, w.blk, m.row_ptr, m.col_idx)
+    dt = time.perf_counter() - t0
+    sub = W.Workload(**{**w.__dict__, "H": heads})
+    return dt, block_flops(sub, m.row_ptr, m.col_idx)
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = workload(args.workload)
+    if w.source != "asa":
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "the CPU oracle arm times the ASA workloads only"}), flush=True)
+        return
+    heads = max(1, min(w.H, args.ref_heads_per_step))
+    qkv = oracle_inputs(w, heads)
+    for _ in range(args.warmup):
+        oracle_step(w, qkv, heads)
+    times, fl = [], 0.0
+    for _ in range(args.steps):
+        dt, fl = oracle_step(w, qkv, heads)
+        times.append(dt)
+    sec = sum(times) / len(times)
+    val = fl / sec / 1e12
+    sample = (f"{w.name}: heads 0..{heads - 1} of {w.H} per step "
+              f"(ASA mask + masked attention, fp64 numpy)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOPS",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "blk": w.blk,
+                   "sample_heads": heads},
+        "cpu_baseline": {"value": val, "unit": "TFLOPS", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU
+def run_gpu(args, rank, world, local):
+    from block_sparse_attention_asa_b200 import bsa
+    w = workload(args.workload)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    q_h, k_h, v_h = W.make_qkv(w)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    B, H, N, d = q.shape
+    nb = w.nb
+    rows = B * H * nb
+    if w.source == "asa":
+        cap = bsa.asa_max_nnz(B, H, N, w.blk, w.mode, w.topk, w.max_keep_ratio, w.keep_diag,
+                              w.n_sink_blocks)
+        ws = torch.empty(bsa.asa_workspace_size(B, H, N, d, w.blk), dtype=torch.uint8, device=dev)
+    else:
+        _, ci_probe = bsa.pattern_mask(w.head_pattern, B, H, N, w.blk, w.band_w, w.frame_tokens,
+                                       w.f_lo, w.f_hi, w.stripe_blocks, w.tile_global_frames,
+                                       device=dev)
+        cap = int(ci_probe.numel())
+        ws = None
+    row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    hp = None
+    if w.source == "pattern":
+        import ctypes
+        hp = (ctypes.c_int32 * H)(*w.head_pattern)
+
+    def mask():
+        if w.source == "asa":
+            bsa.asa_build_mask_into(q, k, w.blk, w.mode, w.topk, w.mass_tau, w.max_keep_ratio,
+                                    w.keep_diag, w.n_sink_blocks, 0.0, row_ptr, col_idx, ws)
+        else:
+            bsa.pattern_mask_into(hp, B, H, N, w.blk, w.band_w, w.frame_tokens, w.f_lo, w.f_hi,
+                                  w.stripe_blocks, w.tile_global_frames, row_ptr, col_idx)
+
+    def forward():
+        bsa.bsa_forward_into(q, k, v, w.blk, row_ptr, col_idx, o, lse)
+
+    launches_per_step = (4 if w.source == "asa" else 3) + 1
+    for _ in range(args.warmup):
+        mask()
+        forward()
+    st = bsa.check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {bsa.status_string(st)}")
+    rp_h = row_ptr.cpu().numpy()
+    ci_h = col_idx[:int(rp_h[-1])].cpu().numpy()
+    flops = block_flops(w, rp_h, ci_h)
+    keep = float(rp_h[-1]) / (rows * nb)
+
+    # ---- timed region: K steps, per-kernel events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_all0 = torch.cuda.Event(enable_timing=True)
+        t_all1 = torch.cuda.Event(enable_timing=True)
+        t_all0.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            mask()
+            ev[s][1].record(stream)
+            forward()
+            ev[s][2].record(stream)
+        t_all1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = t_all0.elapsed_time(t_all1)
+    mask_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    fwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = barrier_max(total_ms, world)
+    ms_step = total_ms / args.steps
+    st = bsa.check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {bsa.status_string(st)}")
+
+    # ---- end to end through the public API with host buffers (pinned), copies timed
+    q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
+    o_p = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    e2e_steps = max(1, min(args.steps, 20))
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        q.copy_(q_p, non_blocking=True)
+        k.copy_(k_p, non_blocking=True)
+        v.copy_(v_p, non_blocking=True)
+        mask()
+        forward()
+        o_p.copy_(o, non_blocking=True)
+        lse_p.copy_(lse, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = barrier_max(e0.elapsed_time(e1) / e2e_steps, world)
+    h2d = 3 * q.numel() * q.element_size()
+    d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
+
+    pk, pk_kind = peaks()
+    fwd_avg = statistics.mean(fwd_ms)
+    mask_avg = statistics.mean(mask_ms)
+    achieved = flops / (fwd_avg * 1e-3) / 1e12
+    peak = float(pk["bf16_tflops"])
+    mask_bytes = (2.0 * q.numel() * 2 + 4.0 * (rows + 1) + 4.0 * rp_h[-1]) if w.source == "asa" \
+        else (4.0 * (rows + 1) + 4.0 * rp_h[-1])
+    mask_gbs = mask_bytes / (mask_avg * 1e-3) / 1e9
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {
+            "workload": w.name, "B": B, "H": H, "N": N, "d": d, "blk": w.blk,
+            "mask": (f"mass tau={w.mass_tau} cap={w.max_keep_ratio}" if w.source == "asa" and
+                     w.mode == W.MODE_MASS else
+                     f"topk k={w.topk} sink={w.n_sink_blocks} diag={w.keep_diag}"
+                     if w.source == "asa" else "fixed patterns per head"),
+            "keep_ratio": keep, "block_flops": flops,
+            "l2": f"inputs larger than L2: Q+K+V = {3 * q.numel() * 2 / 1e6:.0f} MB per step",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+        },
+        "ms_mask": mask_avg, "ms_forward": fwd_avg,
+        "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_kind": f"{pk_kind} bf16 burst", "traffic": None,
+                     "frac_of_sustained": achieved / float(pk.get("bf16_tflops_sustained", peak)),
+                     "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS},
+        "mask_roofline": {"bound": "hbm", "achieved": mask_gbs, "peak": float(pk["hbm_gbs"]),
+                          "unit": "GB/s", "frac": mask_gbs / float(pk["hbm_gbs"]),
+                          "frac_of_8tbs": mask_gbs / DATASHEET_HBM_GBS},
+        "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "clocks": clk.summary(),
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.source == "asa":
+        heads = max(1, min(w.H, args.ref_heads))
+        dt, fl = oracle_step(w, oracle_inputs(w, heads), heads)
+        out["cpu_baseline"] = {"value": fl / dt / 1e12, "unit": "TFLOPS", "cores": os.cpu_count(),
+                               "kind": "oracle",
+                               "sample": f"heads 0..{heads - 1} of {w.H}, one pass, "
+                                         f"{dt:.1f} s fp64 numpy"}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="bsa", choices=["bsa", "reference"])
+    ap.add_argument("--workload", default="wan", choices=["wan", "cog", "hunyuan", "tiny"])
+    ap.add_argument("--ref-heads", type=int, default=6,
+                    help="heads in the cpu_baseline sample of the GPU arm")
+    ap.add_argument("--ref-heads-per-step", type=int, default=1,
+                    help="heads per step of the --impl reference arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_gpu(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

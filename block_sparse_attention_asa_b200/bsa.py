@@ -1,0 +1,231 @@
+"""Python binding of libbsa_b200.so (include/bsa.h), over ctypes.
+
+Argument marshalling only: torch provides device memory and the current
+stream; every step of the computation runs in the library's CUDA kernels.
+There is no fallback: without the built library, or without a CUDA device,
+the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsa_b200.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "bsa.h")
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED = -2
+ERR_CAPACITY = -3
+ERR_CUDA = -4
+ERR_TIMEOUT = -5
+ERR_CSR = -6
+ERR_WORKSPACE = -7
+
+MODE_TOPK = 0
+MODE_MASS = 1
+
+_c_int, _c_float, _c_size, _c_i64, _vp = (ctypes.c_int, ctypes.c_float, ctypes.c_size_t,
+                                          ctypes.c_int64, ctypes.c_void_p)
+
+_SIGNATURES = {
+    "asa_build_mask_workspace_size": (_c_size, [_c_int] * 5),
+    "asa_build_mask_max_nnz": (_c_i64, [_c_int] * 6 + [_c_float, _c_int, _c_int]),
+    "asa_build_mask": (_c_int, [_vp, _vp] + [_c_int] * 7 + [_c_float, _c_float, _c_int, _c_int,
+                                                             _c_float, _vp, _vp, _c_i64, _vp,
+                                                             _c_size, _vp]),
+    "pattern_mask": (_c_int, [_vp] + [_c_int] * 10 + [_vp, _vp, _c_i64, _vp, _vp]),
+    "bsa_forward_workspace_size": (_c_size, [_c_int] * 5),
+    "bsa_forward": (_c_int, [_vp, _vp, _vp] + [_c_int] * 5 + [_vp, _vp, _c_float, _vp, _vp, _vp,
+                                                              _c_size, _vp]),
+    "bsa_check_device_status": (_c_int, [_vp]),
+    "bsa_status_string": (ctypes.c_char_p, [_c_int]),
+    "bsa_version": (_c_int, []),
+}
+
+_lib = None
+
+
+class BsaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} ({code})")
+
+
+def header_functions() -> list:
+    """Names of the functions include/bsa.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b([a-z_][a-z0-9_]*)\s*\(",
+                                 text, flags=re.M)))
+
+
+def load(path: str = LIB_PATH):
+    """Load the library (once) and declare every exported signature."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"libbsa_b200.so is not built ({path}); run "
+                           "block_sparse_attention_asa_b200/build.py")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().bsa_status_string(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise BsaError(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if not (isinstance(t, torch.Tensor) and t.is_cuda and t.is_contiguous()):
+            raise ValueError("expected contiguous CUDA tensors")
+
+
+def _shape(q: torch.Tensor):
+    if q.dim() != 4 or q.dtype != torch.bfloat16:
+        raise ValueError("q/k/v must be bf16 [B, H, N, d]")
+    return tuple(int(x) for x in q.shape)
+
+
+def check_device_status(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device status word."""
+    return int(load().bsa_check_device_status(_stream(stream)))
+
+
+# ----------------------------------------------------------------------------- ASA
+def asa_workspace_size(B: int, H: int, N: int, d: int, blk: int) -> int:
+    return int(load().asa_build_mask_workspace_size(B, H, N, d, blk))
+
+
+def asa_max_nnz(B, H, N, blk, mode, topk=0, max_keep_ratio=0.0, keep_diag=0, n_sink_blocks=0) -> int:
+    return int(load().asa_build_mask_max_nnz(B, H, N, blk, mode, topk, max_keep_ratio, keep_diag,
+                                            n_sink_blocks))
+
+
+def asa_build_mask_into(q, k, blk, mode, topk, mass_tau, max_keep_ratio, keep_diag, n_sink_blocks,
+                        softmax_scale, row_ptr, col_idx, workspace, stream=None):
+    """Raw call into preallocated outputs; asynchronous, no allocation, no sync."""
+    B, H, N, d = _shape(q)
+    lib = load()
+    rc = lib.asa_build_mask(_ptr(q), _ptr(k), B, H, N, d, blk, mode, topk, mass_tau,
+                            max_keep_ratio, keep_diag, n_sink_blocks, softmax_scale, _ptr(row_ptr),
+                            _ptr(col_idx), col_idx.numel(), _ptr(workspace),
+                            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(rc, "asa_build_mask")
+
+
+def asa_build_mask(q: torch.Tensor, k: torch.Tensor, blk: int, mode: int = MODE_TOPK, topk: int = 0,
+                   mass_tau: float = 0.0, max_keep_ratio: float = 0.0, keep_diag: int = 0,
+                   n_sink_blocks: int = 0, softmax_scale: float = 0.0, trim: bool = True,
+                   stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """CSR (row_ptr, col_idx) of the ASA mask.  trim=True reads nnz back (syncs)."""
+    _need_cuda(q, k)
+    B, H, N, d = _shape(q)
+    nb = -(-N // blk)
+    dev = q.device
+    cap = asa_max_nnz(B, H, N, blk, mode, topk, max_keep_ratio, keep_diag, n_sink_blocks)
+    if cap < 0:
+        raise BsaError(ERR_UNSUPPORTED, "asa_build_mask")
+    row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    ws = torch.empty(max(asa_workspace_size(B, H, N, d, blk), 256), dtype=torch.uint8, device=dev)
+    asa_build_mask_into(q, k, blk, mode, topk, mass_tau, max_keep_ratio, keep_diag, n_sink_blocks,
+                        softmax_scale, row_ptr, col_idx, ws, stream)
+    if trim:
+        nnz = int(row_ptr[-1].item())
+        col_idx = col_idx[:nnz]
+    return row_ptr, col_idx
+
+
+# ----------------------------------------------------------------------------- patterns
+def pattern_mask(head_pattern: Sequence[int], B: int, H: int, N: int, blk: int, band_w: int = 2,
+                 frame_tokens: int = 1, f_lo: int = 0, f_hi: int = 0, stripe_blocks: int = 0,
+                 tile_global_frames: int = 0, device=None, stream=None):
+    """CSR of the per-head fixed patterns (syncs once to size col_idx)."""
+    lib = load()
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    nb = -(-N // blk)
+    hp = (ctypes.c_int32 * H)(*[int(x) for x in head_pattern])
+    row_ptr = torch.empty(B * H * nb + 1, dtype=torch.int32, device=dev)
+    nnz = ctypes.c_int64(0)
+    # first pass with zero capacity: counts, scan and the nnz (writes nothing)
+    rc = lib.pattern_mask(hp, B, H, N, blk, band_w, frame_tokens, f_lo, f_hi, stripe_blocks,
+                          tile_global_frames, _ptr(row_ptr), None, 0, ctypes.byref(nnz),
+                          _stream(stream))
+    if rc not in (OK, ERR_CAPACITY):
+        _check(rc, "pattern_mask")
+    col_idx = torch.empty(max(int(nnz.value), 1), dtype=torch.int32, device=dev)
+    pattern_mask_into(hp, B, H, N, blk, band_w, frame_tokens, f_lo, f_hi, stripe_blocks,
+                      tile_global_frames, row_ptr, col_idx, stream)
+    return row_ptr, col_idx[:int(nnz.value)]
+
+
+def pattern_mask_into(head_pattern, B, H, N, blk, band_w, frame_tokens, f_lo, f_hi, stripe_blocks,
+                      tile_global_frames, row_ptr, col_idx, stream=None):
+    """Raw asynchronous call into preallocated outputs."""
+    lib = load()
+    if not isinstance(head_pattern, ctypes.Array):
+        head_pattern = (ctypes.c_int32 * H)(*[int(x) for x in head_pattern])
+    rc = lib.pattern_mask(head_pattern, B, H, N, blk, band_w, frame_tokens, f_lo, f_hi,
+                          stripe_blocks, tile_global_frames, _ptr(row_ptr), _ptr(col_idx),
+                          col_idx.numel(), None, _stream(stream))
+    _check(rc, "pattern_mask")
+
+
+# ----------------------------------------------------------------------------- forward
+def bsa_forward_into(q, k, v, blk, row_ptr, col_idx, o, lse=None, softmax_scale=0.0,
+                     workspace=None, stream=None):
+    B, H, N, d = _shape(q)
+    lib = load()
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib.bsa_forward(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, blk, _ptr(row_ptr), _ptr(col_idx),
+                         softmax_scale, _ptr(o), _ptr(lse), _ptr(workspace), ws_bytes,
+                         _stream(stream))
+    _check(rc, "bsa_forward")
+
+
+def bsa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blk: int, row_ptr: torch.Tensor,
+                col_idx: torch.Tensor, softmax_scale: float = 0.0, stream=None):
+    """(O bf16 [B,H,N,d], LSE fp32 [B,H,N]) of attention over the CSR's kept blocks."""
+    _need_cuda(q, k, v, row_ptr)
+    B, H, N, d = _shape(q)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    ws_n = int(load().bsa_forward_workspace_size(B, H, N, d, blk))
+    ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
+    if col_idx.numel() == 0:
+        col_idx = torch.zeros(1, dtype=torch.int32, device=q.device)
+    bsa_forward_into(q, k, v, blk, row_ptr, col_idx, o, lse, softmax_scale, ws, stream)
+    return o, lse
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,351 @@
+// asa_mask.cuh -- BLADE's Adaptive Block-Sparse Attention mask on sm_100a.
+//
+// BLADE digest (abstract; 方法详解 / 关键设计): ASA builds, per input, a mask that
+// keeps the block pairs whose mutual relevance is high.  Reading used here
+// (documented in include/bsa.h): mean-pool Q and K per token block, softmax of
+// the pooled scores over all kv-blocks, keep by top-k or by the shortest prefix
+// reaching a cumulative mass, ties to the lower block index, optional cap and
+// forced blocks, CSR out.
+//
+// Kernels, in launch order:
+//   asa_pool_kernel    HBM-bound: streams Q and K once (16-byte loads, fp32
+//                      accumulation in a fixed order), writes q̄, k̄ fp32.
+//   asa_select_kernel  per CTA: R q-block rows of one (b, h).  Scores against
+//                      all k̄ (staged through shared memory), softmax, then a
+//                      per-row radix select on the order key
+//                      (p desc, j asc) -> selection bitmap and count.
+//   csr_scan_kernel    counts -> row_ptr.
+//   asa_expand_kernel  bitmaps -> ascending col_idx.
+#pragma once
+#include "common.cuh"
+#include <cuda_bf16.h>
+
+namespace bsa {
+
+// ------------------------------------------------------------------ pooling
+// One warp per (tensor, b, h, block).  Lane l reads 16 bytes (8 elements) of a
+// row; D/8 lanes cover a row, 256/D rows per warp step.
+template <int D>
+__global__ void __launch_bounds__(256) asa_pool_kernel(const __nv_bfloat16* __restrict__ q,
+                                                       const __nv_bfloat16* __restrict__ k,
+                                                       float* __restrict__ pooled, int BH, int N,
+                                                       int blk, int nb) {
+  constexpr int LPR = D / 8;          // lanes per row
+  constexpr int RPS = 32 / LPR;       // rows per warp step
+  const int lane = threadIdx.x & 31;
+  const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const long long units = 2LL * BH * nb;
+  if (unit >= units) return;
+  const bool is_k = unit >= (long long)BH * nb;
+  const long long u = is_k ? unit - (long long)BH * nb : unit;
+  const long long bh = u / nb;
+  const int i = static_cast<int>(u % nb);
+  const int r0 = i * blk, nrows = min(blk, N - r0);
+  const __nv_bfloat16* src = (is_k ? k : q) + (bh * N + r0) * D;
+  const int sub = lane / LPR, col = (lane % LPR) * 8;
+  float acc[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) acc[c] = 0.f;
+#pragma unroll 4
+  for (int r = sub; r < nrows; r += RPS) {
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + (long long)r * D + col));
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float2 f = __bfloat1622float2(h2[c]);
+      acc[2 * c] += f.x;
+      acc[2 * c + 1] += f.y;
+    }
+  }
+  // combine the row groups (fixed butterfly order)
+#pragma unroll
+  for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
+  if (sub == 0) {
+    const float n = static_cast<float>(nrows);
+    float4 a, b;
+    a.x = acc[0] / n; a.y = acc[1] / n; a.z = acc[2] / n; a.w = acc[3] / n;
+    b.x = acc[4] / n; b.y = acc[5] / n; b.z = acc[6] / n; b.w = acc[7] / n;
+    float* dst = pooled + unit * D + col;
+    reinterpret_cast<float4*>(dst)[0] = a;
+    reinterpret_cast<float4*>(dst)[1] = b;
+  }
+}
+
+// ------------------------------------------------------------------ select
+struct SelectParams {
+  const float* qbar;      // [BH*nb, D]
+  const float* kbar;      // [BH*nb, D]
+  uint32_t* bitmaps;      // [BH*nb, nbw]
+  int32_t* row_ptr;       // counts go to row_ptr[r+1]
+  int nb, nbw, rows_per_cta, nb_pad;
+  int mode, topk, cap, keep_diag, n_sink;
+  float mass_tau, scale;
+};
+
+constexpr int kSelWarps = 8;
+constexpr int kKChunk = 64;
+
+// Order key: ascending key <=> (p descending, j ascending).  p >= 0, so its
+// bit pattern orders like its value.
+__device__ __forceinline__ unsigned long long order_key(float p, int j) {
+  return (static_cast<unsigned long long>(0xFFFFFFFFu - __float_as_uint(p)) << 32) |
+         static_cast<unsigned int>(j);
+}
+
+// The m-th smallest order key (1-based m, 1 <= m <= nb <= 65536) of the row
+// `pr`, by an 8-bit-digit radix select over the key's significant bytes: the
+// four bytes of the p bits, then -- only while elements with equal p remain to
+// be split -- the two low bytes of the block index.
+__device__ unsigned long long kth_key(const float* pr, int nb, int m, unsigned int* hist) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long prefix = 0, pmask = 0;
+  int remaining = m;
+#pragma unroll 1
+  for (int pass = 0; pass < 6; ++pass) {
+    const int shift = pass < 4 ? 56 - 8 * pass : (pass == 4 ? 8 : 0);
+    if (pass == 4) {
+      // p settled; if exactly `remaining` elements carry it, take them all
+      int eq = 0, last = -1;
+      for (int j = lane; j < nb; j += 32)
+        if ((order_key(pr[j], j) & pmask) == prefix) {
+          ++eq;
+          last = j;
+        }
+      eq = warp_sum(eq);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+      if (eq == remaining) return prefix | static_cast<unsigned int>(last);
+    }
+#pragma unroll
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int j = lane; j < nb; j += 32) {
+      const unsigned long long key = order_key(pr[j], j);
+      if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+    }
+    __syncwarp();
+    // lane owns bins [8*lane, 8*lane+8), ascending digit order
+    int mine = 0;
+#pragma unroll
+    for (int b = 0; b < 8; ++b) mine += hist[8 * lane + b];
+    const int incl = warp_incl_scan(mine);
+    const int excl = incl - mine;
+    const unsigned who = __ballot_sync(0xffffffffu, excl < remaining && remaining <= incl);
+    const int src = __ffs(who) - 1;
+    int digit = 0, below = 0;
+    if (lane == src) {
+      int c = excl;
+      for (int b = 0; b < 8; ++b) {
+        const int hb = hist[8 * lane + b];
+        if (c + hb >= remaining) {
+          digit = 8 * lane + b;
+          below = c;
+          break;
+        }
+        c += hb;
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    below = __shfl_sync(0xffffffffu, below, src);
+    __syncwarp();
+    remaining -= below;
+    prefix |= static_cast<unsigned long long>(digit) << shift;
+    pmask |= 0xFFull << shift;
+  }
+  return prefix;
+}
+
+// Number of blocks the mass rule keeps: the shortest prefix (in key order)
+// whose p sum reaches tau, looked for in chunks of 64 ranks, at most `limit`.
+__device__ int mass_count(const float* pr, int nb, float tau, int limit, unsigned int* hist,
+                          unsigned long long* buf) {
+  const int lane = threadIdx.x & 31;
+  float total = 0.f;
+  unsigned long long k_lo = 0;  // keys <= k_lo are already counted
+  bool have_lo = false;
+#pragma unroll 1
+  for (int done = 0; done < limit; done += 64) {
+    const int upto = min(limit, done + 64);
+    const unsigned long long k_hi = kth_key(pr, nb, upto, hist);
+    // gather keys in (k_lo, k_hi]
+    int n = 0;
+    for (int jb = 0; jb < nb; jb += 32) {
+      const int j = jb + lane;
+      unsigned long long key = 0;
+      bool in = false;
+      if (j < nb) {
+        key = order_key(pr[j], j);
+        in = key <= k_hi && (!have_lo || key > k_lo);
+      }
+      const unsigned msk = __ballot_sync(0xffffffffu, in);
+      if (in) buf[n + __popc(msk & ((1u << lane) - 1u))] = key;
+      n += __popc(msk);
+    }
+    __syncwarp();
+    // bitonic sort of 64 keys, element x = lane + 32*h
+    unsigned long long e0 = lane < n ? buf[lane] : ~0ull;
+    unsigned long long e1 = lane + 32 < n ? buf[lane + 32] : ~0ull;
+    __syncwarp();
+#pragma unroll
+    for (int kk = 2; kk <= 64; kk <<= 1) {
+#pragma unroll
+      for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+        if (jj == 32) {
+          // partner is the other register of the same lane (x and x+32)
+          const bool asc = ((lane & kk) == 0);  // kk == 64 here: always ascending
+          const unsigned long long lo = e0 < e1 ? e0 : e1, hi = e0 < e1 ? e1 : e0;
+          e0 = asc ? lo : hi;
+          e1 = asc ? hi : lo;
+        } else {
+          const unsigned long long p0 = __shfl_xor_sync(0xffffffffu, e0, jj);
+          const unsigned long long p1 = __shfl_xor_sync(0xffffffffu, e1, jj);
+          const bool lower = (lane & jj) == 0;
+          const bool asc0 = ((lane & kk) == 0);
+          const bool asc1 = (((lane + 32) & kk) == 0);
+          e0 = (lower == asc0) ? (e0 < p0 ? e0 : p0) : (e0 < p0 ? p0 : e0);
+          e1 = (lower == asc1) ? (e1 < p1 ? e1 : p1) : (e1 < p1 ? p1 : e1);
+        }
+      }
+    }
+    // p in sorted order; padding keys decode to p = 0
+    const float p0 = __uint_as_float(0xFFFFFFFFu - static_cast<unsigned int>(e0 >> 32));
+    const float p1 = __uint_as_float(0xFFFFFFFFu - static_cast<unsigned int>(e1 >> 32));
+    const float s0 = warp_incl_scan_f(p0);
+    const float t0 = __shfl_sync(0xffffffffu, s0, 31);
+    const float s1 = warp_incl_scan_f(p1) + t0;
+    const unsigned hit0 = __ballot_sync(0xffffffffu, lane < n && total + s0 >= tau);
+    const unsigned hit1 = __ballot_sync(0xffffffffu, lane + 32 < n && total + s1 >= tau);
+    if (hit0) return done + __ffs(hit0);
+    if (hit1) return done + 32 + __ffs(hit1);
+    total += __shfl_sync(0xffffffffu, s1, 31);
+    k_lo = k_hi;
+    have_lo = true;
+  }
+  return limit;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) asa_select_kernel(const SelectParams p) {
+  extern __shared__ __align__(16) unsigned char sel_smem[];
+  const int R = p.rows_per_cta;
+  float* qs = reinterpret_cast<float*>(sel_smem);                  // [R][D]
+  float* kc = qs + R * D;                                          // [64][D+1]
+  float* sc = kc + kKChunk * (D + 1);                              // [R][nb_pad]
+  unsigned int* hist = reinterpret_cast<unsigned int*>(sc + (size_t)R * p.nb_pad);  // [8][256]
+  unsigned long long* buf =
+      reinterpret_cast<unsigned long long*>(hist + kSelWarps * 256);  // [8][64]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.y, i0 = blockIdx.x * R;
+  const int nrow = min(R, p.nb - i0);
+  const float* qrow = p.qbar + ((long long)bh * p.nb + i0) * D;
+  const float* kbh = p.kbar + (long long)bh * p.nb * D;
+
+  for (int e = tid; e < nrow * D; e += 256) qs[e] = qrow[e];
+  // scores: thread (ty, tx) -> row ty, columns tx + 16*m of the chunk
+  const int ty = tid >> 4, tx = tid & 15;
+  for (int jc = 0; jc < p.nb; jc += kKChunk) {
+    __syncthreads();
+    const int nj = min(kKChunk, p.nb - jc);
+    for (int e = tid; e < nj * D; e += 256) {
+      const int jj = e / D, dd = e % D;
+      kc[jj * (D + 1) + dd] = kbh[(long long)(jc + jj) * D + dd];
+    }
+    __syncthreads();
+    for (int rr = ty; rr < nrow; rr += 16) {
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const float* qv = qs + rr * D;
+#pragma unroll 8
+      for (int dd = 0; dd < D; ++dd) {
+        const float a = qv[dd];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) acc[m] = fmaf(a, kc[(tx + 16 * m) * (D + 1) + dd], acc[m]);
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int jj = tx + 16 * m;
+        if (jj < nj) sc[rr * p.nb_pad + jc + jj] = acc[m] * p.scale;
+      }
+    }
+  }
+  __syncthreads();
+
+  unsigned int* myhist = hist + warp * 256;
+  unsigned long long* mybuf = buf + warp * 64;
+  for (int rr = warp; rr < nrow; rr += kSelWarps) {
+    float* pr = sc + rr * p.nb_pad;
+    const int i = i0 + rr;
+    // softmax over all nb blocks (fixed reduction order)
+    float mx = -INFINITY;
+    for (int j = lane; j < p.nb; j += 32) mx = fmaxf(mx, pr[j]);
+    mx = warp_max(mx);
+    float sum = 0.f;
+    for (int j = lane; j < p.nb; j += 32) {
+      const float e = expf(pr[j] - mx);
+      pr[j] = e;
+      sum += e;
+    }
+    sum = warp_sum_f(sum);
+    for (int j = lane; j < p.nb; j += 32) pr[j] = pr[j] / sum;
+    __syncwarp();
+    int m;
+    if (p.mode == BSA_MODE_TOPK) {
+      m = min(min(p.topk, p.cap), p.nb);
+    } else {
+      m = mass_count(pr, p.nb, p.mass_tau, min(p.cap, p.nb), myhist, mybuf);
+    }
+    const unsigned long long kth = kth_key(pr, p.nb, m, myhist);
+    const long long r = (long long)bh * p.nb + i;
+    uint32_t* dst = p.bitmaps + r * p.nbw;
+    int cnt = 0;
+    for (int wd = 0; wd < p.nbw; ++wd) {
+      const int j = wd * 32 + lane;
+      bool keep = false;
+      if (j < p.nb) {
+        keep = order_key(pr[j], j) <= kth;
+        if (p.keep_diag && j == i) keep = true;
+        if (j < p.n_sink) keep = true;
+      }
+      const unsigned word = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0) dst[wd] = word;
+      cnt += __popc(word);
+    }
+    if (lane == 0) p.row_ptr[r + 1] = cnt;
+    __syncwarp();
+  }
+}
+
+// ------------------------------------------------------------------ expand
+// One warp per row: set bits of the row's bitmap -> ascending block ids.
+__global__ void __launch_bounds__(256) asa_expand_kernel(const uint32_t* __restrict__ bitmaps,
+                                                         const int32_t* __restrict__ row_ptr,
+                                                         int32_t* __restrict__ col_idx,
+                                                         long long capacity, long long rows,
+                                                         int nbw) {
+  const int lane = threadIdx.x & 31;
+  const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  long long pos = row_ptr[r];
+  const uint32_t* bmr = bitmaps + r * nbw;
+  for (int w0 = 0; w0 < nbw; w0 += 32) {
+    const int wd = w0 + lane;
+    uint32_t word = wd < nbw ? bmr[wd] : 0u;
+    const int c = __popc(word);
+    const int incl = warp_incl_scan(c);
+    long long at = pos + incl - c;
+    while (word) {
+      const int bit = __ffs(word) - 1;
+      word &= word - 1;
+      if (at < capacity)
+        col_idx[at] = wd * 32 + bit;
+      else
+        record_error(BSA_ERR_CAPACITY);
+      ++at;
+    }
+    pos += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+}  // namespace bsa

@@ -1,0 +1,376 @@
+// bsa_api.cu -- the C ABI of include/bsa.h: host-side validation, TMA tensor
+// maps and kernel launches.  Every compute step runs in the kernels included
+// below; this file only checks arguments, sizes grids and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/bsa.h"
+#include "common.cuh"
+#include "pattern.cuh"
+#include "asa_mask.cuh"
+#include "bsa_fwd.cuh"
+
+namespace {
+
+using bsa::FwdCfg;
+
+constexpr unsigned long long kWaitNs = 1000000000ull;  // 1 s bound on device waits
+
+inline cudaStream_t as_cuda(bsa_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+inline int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline bool blk_ok(int blk) { return blk == 16 || blk == 32 || blk == 64 || blk == 128; }
+
+inline int check_launch() { return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+int common_shape_checks(int B, int H, int N, int blk) {
+  if (B <= 0 || H <= 0 || N <= 0 || blk <= 0) return BSA_ERR_INVALID_ARG;
+  if (!blk_ok(blk)) return BSA_ERR_UNSUPPORTED;
+  const long long nb = (N + blk - 1) / blk;
+  if ((long long)B * H * nb * nb >= (1LL << 31)) return BSA_ERR_UNSUPPORTED;
+  if ((long long)B * H > 65535) return BSA_ERR_UNSUPPORTED;  // grid.y
+  return BSA_OK;
+}
+
+// ---- tensor maps ------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [B*H, N, d] bf16 viewed as a 3D tensor {d, N, B*H}; box {64, rows, 1}, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---- forward launch -----------------------------------------------------------
+template <int D, int BLK>
+int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
+               const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o, float* lse,
+               cudaStream_t stream) {
+  using C = FwdCfg<D, BLK>;
+  const int nb = (N + BLK - 1) / BLK;
+  const int nbw = (nb + 31) / 32;
+  if ((long long)C::QB * nbw * 4 > C::kMaxBitmapBytes) return BSA_ERR_UNSUPPORTED;
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, B * H, N, D, 128) || !make_map(&mk, k, B * H, N, D, BLK) ||
+      !make_map(&mv, v, B * H, N, D, BLK))
+    return BSA_ERR_CUDA;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_set[dev]) {
+    if (cudaFuncSetAttribute(bsa::bsa_fwd_kernel<D, BLK>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+      return BSA_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  bsa::FwdParams p;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.nb = nb;
+  p.nbw = nbw;
+  p.nqt = ceil_div(N, 128);
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.wait_ns = kWaitNs;
+  dim3 grid(p.nqt, B * H);
+  bsa::bsa_fwd_kernel<D, BLK><<<grid, 256, C::SMEM, stream>>>(mq, mk, mv, p);
+  return check_launch();
+}
+
+template <int D>
+int launch_fwd_blk(int blk, const void* q, const void* k, const void* v, int B, int H, int N,
+                   const int32_t* rp, const int32_t* ci, float scale, void* o, float* lse,
+                   cudaStream_t s) {
+  switch (blk) {
+    case 16: return launch_fwd<D, 16>(q, k, v, B, H, N, rp, ci, scale, o, lse, s);
+    case 32: return launch_fwd<D, 32>(q, k, v, B, H, N, rp, ci, scale, o, lse, s);
+    case 64: return launch_fwd<D, 64>(q, k, v, B, H, N, rp, ci, scale, o, lse, s);
+    case 128: return launch_fwd<D, 128>(q, k, v, B, H, N, rp, ci, scale, o, lse, s);
+  }
+  return BSA_ERR_UNSUPPORTED;
+}
+
+// ---- ASA mask sizes -------------------------------------------------------------
+struct AsaLayout {
+  long long nb, nbw, rows;
+  size_t pooled_bytes, bitmap_bytes, total;
+};
+
+AsaLayout asa_layout(int B, int H, int N, int d, int blk) {
+  AsaLayout L;
+  L.nb = (N + blk - 1) / blk;
+  L.nbw = (L.nb + 31) / 32;
+  L.rows = (long long)B * H * L.nb;
+  L.pooled_bytes = (size_t)2 * L.rows * d * sizeof(float);
+  L.bitmap_bytes = (size_t)L.rows * L.nbw * sizeof(uint32_t);
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  L.total = up(L.pooled_bytes) + up(L.bitmap_bytes);
+  return L;
+}
+
+int select_cap(int nb, float ratio) {
+  if (!(ratio > 0.f)) return nb;
+  const int c = static_cast<int>(std::floor(static_cast<double>(ratio) * nb));
+  return c < 1 ? 1 : (c > nb ? nb : c);
+}
+
+template <int D>
+size_t select_smem(int R, int nb_pad, int nbw) {
+  (void)nbw;
+  return (size_t)R * D * 4 + (size_t)bsa::kKChunk * (D + 1) * 4 + (size_t)R * nb_pad * 4 +
+         (size_t)bsa::kSelWarps * 256 * 4 + (size_t)bsa::kSelWarps * 64 * 8;
+}
+
+template <int D>
+int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int mode, int topk,
+               float tau, float ratio, int keep_diag, int n_sink, float scale, int32_t* row_ptr,
+               int32_t* col_idx, long long cap_entries, void* ws, cudaStream_t stream) {
+  const AsaLayout L = asa_layout(B, H, N, D, blk);
+  const int nb = static_cast<int>(L.nb), nbw = static_cast<int>(L.nbw);
+  const int BH = B * H;
+  float* pooled = static_cast<float*>(ws);
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) +
+                                                  ((L.pooled_bytes + 255) & ~(size_t)255));
+  // 1. pooling
+  {
+    const long long units = 2LL * BH * nb;
+    bsa::asa_pool_kernel<D><<<ceil_div(units, 8), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), pooled, BH, N,
+        blk, nb);
+    if (check_launch()) return BSA_ERR_CUDA;
+  }
+  // 2. scores + selection
+  {
+    const int nb_pad = (nb + 31) / 32 * 32;
+    const size_t budget = 200 * 1024;
+    int R = 16;
+    while (R > 1 && select_smem<D>(R, nb_pad, nbw) > budget) --R;
+    const size_t smem = select_smem<D>(R, nb_pad, nbw);
+    if (smem > budget) return BSA_ERR_UNSUPPORTED;
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr_set[dev]) {
+      if (cudaFuncSetAttribute(bsa::asa_select_kernel<D>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024) !=
+          cudaSuccess)
+        return BSA_ERR_CUDA;
+      attr_set[dev] = true;
+    }
+    bsa::SelectParams sp;
+    sp.qbar = pooled;
+    sp.kbar = pooled + (size_t)BH * nb * D;
+    sp.bitmaps = bitmaps;
+    sp.row_ptr = row_ptr;
+    sp.nb = nb;
+    sp.nbw = nbw;
+    sp.rows_per_cta = R;
+    sp.nb_pad = nb_pad;
+    sp.mode = mode;
+    sp.topk = topk;
+    sp.cap = select_cap(nb, ratio);
+    sp.keep_diag = keep_diag;
+    sp.n_sink = n_sink;
+    sp.mass_tau = tau;
+    sp.scale = scale;
+    dim3 grid(ceil_div(nb, R), BH);
+    bsa::asa_select_kernel<D><<<grid, 256, smem, stream>>>(sp);
+    if (check_launch()) return BSA_ERR_CUDA;
+  }
+  // 3. counts -> row_ptr
+  bsa::csr_scan_kernel<<<1, 1024, 0, stream>>>(row_ptr, static_cast<int>(L.rows));
+  if (check_launch()) return BSA_ERR_CUDA;
+  // 4. bitmaps -> col_idx
+  bsa::asa_expand_kernel<<<ceil_div(L.rows, 8), 256, 0, stream>>>(bitmaps, row_ptr, col_idx,
+                                                                  cap_entries, L.rows, nbw);
+  return check_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+int bsa_version(void) { return 100; }
+
+const char* bsa_status_string(int status) {
+  switch (status) {
+    case BSA_OK: return "ok";
+    case BSA_ERR_INVALID_ARG: return "invalid argument";
+    case BSA_ERR_UNSUPPORTED: return "unsupported shape, block size, head dim or alignment";
+    case BSA_ERR_CAPACITY: return "col_idx capacity too small for the mask";
+    case BSA_ERR_CUDA: return "CUDA runtime or launch error";
+    case BSA_ERR_TIMEOUT: return "a device-side wait gave up";
+    case BSA_ERR_CSR: return "CSR block index outside [0, nb)";
+    case BSA_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+  }
+  return "unknown status";
+}
+
+int bsa_check_device_status(bsa_stream_t stream) {
+  if (cudaStreamSynchronize(as_cuda(stream)) != cudaSuccess) return BSA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, bsa::g_status, sizeof(int)) != cudaSuccess) return BSA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(bsa::g_status, &zero, sizeof(int)) != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  return v;
+}
+
+size_t asa_build_mask_workspace_size(int B, int H, int N, int d, int blk) {
+  if (common_shape_checks(B, H, N, blk) != BSA_OK || (d != 64 && d != 128)) return 0;
+  return asa_layout(B, H, N, d, blk).total;
+}
+
+int64_t asa_build_mask_max_nnz(int B, int H, int N, int blk, int mode, int topk,
+                               float max_keep_ratio, int keep_diag, int n_sink_blocks) {
+  if (common_shape_checks(B, H, N, blk) != BSA_OK) return -1;
+  const long long nb = (N + blk - 1) / blk;
+  long long per = select_cap(static_cast<int>(nb), max_keep_ratio);
+  if (mode == BSA_MODE_TOPK) per = per < topk ? per : topk;
+  if (per < 0) per = 0;
+  per += (keep_diag ? 1 : 0) + (n_sink_blocks > 0 ? n_sink_blocks : 0);
+  if (per > nb) per = nb;
+  return (int64_t)B * H * nb * per;
+}
+
+int asa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int blk, int mode,
+                   int topk, float mass_tau, float max_keep_ratio, int keep_diag,
+                   int n_sink_blocks, float softmax_scale, int32_t* row_ptr, int32_t* col_idx,
+                   int64_t col_capacity, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  if (!q || !k || !row_ptr || (!col_idx && col_capacity > 0) || col_capacity < 0)
+    return BSA_ERR_INVALID_ARG;
+  int rc = common_shape_checks(B, H, N, blk);
+  if (rc != BSA_OK) return rc;
+  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16)) return BSA_ERR_UNSUPPORTED;
+  if (mode != BSA_MODE_TOPK && mode != BSA_MODE_MASS) return BSA_ERR_INVALID_ARG;
+  if (mode == BSA_MODE_TOPK && topk < 1) return BSA_ERR_INVALID_ARG;
+  if (mode == BSA_MODE_MASS && !(mass_tau > 0.f && mass_tau <= 1.f)) return BSA_ERR_INVALID_ARG;
+  if (!(max_keep_ratio <= 1.0f) || std::isnan(softmax_scale)) return BSA_ERR_INVALID_ARG;
+  if (n_sink_blocks < 0) return BSA_ERR_INVALID_ARG;
+  const long long nb = (N + blk - 1) / blk;
+  if (nb > 65536) return BSA_ERR_UNSUPPORTED;
+  const AsaLayout L = asa_layout(B, H, N, d, blk);
+  if (!workspace || ws_bytes < L.total || !aligned(workspace, 256)) return BSA_ERR_WORKSPACE;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
+  cudaStream_t s = as_cuda(stream);
+  if (d == 64)
+    return launch_asa<64>(q, k, B, H, N, blk, mode, topk, mass_tau, max_keep_ratio, keep_diag,
+                          n_sink_blocks, scale, row_ptr, col_idx, col_capacity, workspace, s);
+  return launch_asa<128>(q, k, B, H, N, blk, mode, topk, mass_tau, max_keep_ratio, keep_diag,
+                         n_sink_blocks, scale, row_ptr, col_idx, col_capacity, workspace, s);
+}
+
+int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk, int band_w,
+                 int frame_tokens, int f_lo, int f_hi, int stripe_blocks, int tile_global_frames,
+                 int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                 int64_t* nnz_out_host, bsa_stream_t stream) {
+  if (!head_pattern_host || !row_ptr || col_capacity < 0 || (!col_idx && col_capacity > 0))
+    return BSA_ERR_INVALID_ARG;
+  int rc = common_shape_checks(B, H, N, blk);
+  if (rc != BSA_OK) return rc;
+  if (H > bsa::kMaxPatternHeads) return BSA_ERR_UNSUPPORTED;
+  if (band_w < 0 || frame_tokens <= 0 || f_lo > f_hi || stripe_blocks < 0 ||
+      tile_global_frames < 0)
+    return BSA_ERR_INVALID_ARG;
+  bsa::PatternParams p;
+  std::memset(&p, 0, sizeof(p));
+  for (int h = 0; h < H; ++h) {
+    const int v = head_pattern_host[h];
+    if (v < BSA_PATTERN_FULL || v > BSA_PATTERN_TILE3D) return BSA_ERR_INVALID_ARG;
+    p.head_pattern[h] = static_cast<int8_t>(v);
+  }
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.blk = blk;
+  p.nb = (N + blk - 1) / blk;
+  p.band_w = band_w;
+  p.frame_tokens = frame_tokens;
+  p.f_lo = f_lo;
+  p.f_hi = f_hi;
+  p.stripe_blocks = stripe_blocks;
+  p.tile_global_frames = tile_global_frames;
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.capacity = col_capacity;
+  cudaStream_t s = as_cuda(stream);
+  const long long units = (long long)H * p.nb;
+  const long long rows = (long long)B * H * p.nb;
+  bsa::pattern_kernel<false><<<ceil_div(units, 8), 256, 0, s>>>(p);
+  if (check_launch()) return BSA_ERR_CUDA;
+  bsa::csr_scan_kernel<<<1, 1024, 0, s>>>(row_ptr, static_cast<int>(rows));
+  if (check_launch()) return BSA_ERR_CUDA;
+  if (nnz_out_host) {
+    int32_t nnz = 0;
+    if (cudaMemcpyAsync(&nnz, row_ptr + rows, sizeof(int32_t), cudaMemcpyDeviceToHost, s) !=
+            cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return BSA_ERR_CUDA;
+    *nnz_out_host = nnz;
+    if (nnz > col_capacity) return BSA_ERR_CAPACITY;
+  }
+  bsa::pattern_kernel<true><<<ceil_div(units, 8), 256, 0, s>>>(p);
+  return check_launch();
+}
+
+size_t bsa_forward_workspace_size(int B, int H, int N, int d, int blk) {
+  (void)B; (void)H; (void)N; (void)d; (void)blk;
+  return 0;
+}
+
+int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d, int blk,
+                const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale, void* o,
+                float* lse, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  (void)workspace;
+  (void)ws_bytes;
+  if (!q || !k || !v || !o || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
+  int rc = common_shape_checks(B, H, N, blk);
+  if (rc != BSA_OK) return rc;
+  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16))
+    return BSA_ERR_UNSUPPORTED;
+  if (std::isnan(softmax_scale)) return BSA_ERR_INVALID_ARG;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
+  cudaStream_t s = as_cuda(stream);
+  if (d == 64) return launch_fwd_blk<64>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, s);
+  return launch_fwd_blk<128>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, s);
+}
+
+}  // extern "C"

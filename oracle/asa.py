@@ -65,6 +65,7 @@ class RowSelection:
     p_thr: float          # p of the last block kept by the rule (after the cap)
     mass_at_cut: float    # cumulative p of the kept prefix (before the cap)
     n_selected: int       # blocks kept by the rule (before forcing)
+    mass_before_cut: float = 0.0  # cumulative p of the prefix one shorter
 
 
 def select_row(p_row: np.ndarray, i: int, mode: int, topk: int = 0, mass_tau: float = 0.0,
@@ -75,7 +76,8 @@ def select_row(p_row: np.ndarray, i: int, mode: int, topk: int = 0, mass_tau: fl
     order = np.lexsort((np.arange(nb), -p_row))
     if mode == MODE_TOPK:
         m = min(max(topk, 0), nb)
-        mass = float(np.sum(p_row[order[:m]]))
+        mass = math.fsum(p_row[order[:m]].tolist())
+        before = math.fsum(p_row[order[:max(m - 1, 0)]].tolist())
     elif mode == MODE_MASS:
         ps = p_row[order]
         csum = np.cumsum(ps)
@@ -88,6 +90,7 @@ def select_row(p_row: np.ndarray, i: int, mode: int, topk: int = 0, mass_tau: fl
         while m < nb and prefix(m) < mass_tau:
             m += 1
         mass = prefix(m)
+        before = prefix(m - 1)
     else:
         raise ValueError(f"unknown mode {mode}")
     m = min(m, keep_cap(nb, max_keep_ratio))
@@ -96,7 +99,7 @@ def select_row(p_row: np.ndarray, i: int, mode: int, topk: int = 0, mass_tau: fl
     if keep_diag:
         chosen.add(int(i))
     chosen.update(range(min(max(n_sink_blocks, 0), nb)))
-    return RowSelection(sorted(chosen), p_thr, mass, m)
+    return RowSelection(sorted(chosen), p_thr, mass, m, before)
 
 
 @dataclass
@@ -106,6 +109,7 @@ class MaskInfo:
     p_thr: np.ndarray     # float64 [rows]
     mass_at_cut: np.ndarray  # float64 [rows]
     probs: np.ndarray     # float64 [B, H, nb, nb]
+    mass_before_cut: np.ndarray = None  # float64 [rows]
 
 
 def asa_mask(q: np.ndarray, k: np.ndarray, blk: int, mode: int, topk: int = 0,
@@ -120,6 +124,7 @@ def asa_mask(q: np.ndarray, k: np.ndarray, blk: int, mode: int, topk: int = 0,
     cols = []
     p_thr = np.empty(rows)
     mass = np.empty(rows)
+    before = np.empty(rows)
     r = 0
     for b in range(B):
         for h in range(H):
@@ -130,5 +135,6 @@ def asa_mask(q: np.ndarray, k: np.ndarray, blk: int, mode: int, topk: int = 0,
                 row_ptr[r + 1] = row_ptr[r] + len(sel.cols)
                 p_thr[r] = sel.p_thr
                 mass[r] = sel.mass_at_cut
+                before[r] = sel.mass_before_cut
                 r += 1
-    return MaskInfo(row_ptr, np.asarray(cols, dtype=np.int32), p_thr, mass, p)
+    return MaskInfo(row_ptr, np.asarray(cols, dtype=np.int32), p_thr, mass, p, before)

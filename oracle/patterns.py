@@ -51,7 +51,7 @@ def keep_token_pair(pattern: int, t: int, u: int, blk: int, frame_tokens: int, b
 
 def pattern_row(pattern: int, i: int, nb: int, n: int, blk: int, band_w: int, frame_tokens: int,
                 f_lo: int, f_hi: int, stripe_blocks: int, tile_global_frames: int) -> list:
-    """Kept kv-blocks of q-block i, ascending."""
+    """Kept kv-blocks of q-block i, ascending (the rule evaluated for all j at once)."""
     S = frame_tokens
     if pattern == FULL:
         return list(range(nb))
@@ -60,27 +60,26 @@ def pattern_row(pattern: int, i: int, nb: int, n: int, blk: int, band_w: int, fr
     if pattern == DIAG:
         return list(range(max(0, i - band_w), min(nb, i + band_w + 1)))
     ti_lo, ti_hi = _span(i, blk, n)
-    out = []
-    for j in range(nb):
-        uj_lo, uj_hi = _span(j, blk, n)
-        if pattern == MULTIDIAG:
-            # offsets u - t over the two blocks form the integer interval [lo, hi]
-            lo, hi = uj_lo - ti_hi, uj_hi - ti_lo
-            keep = any(lo <= f * S + band_w * blk and hi >= f * S - band_w * blk
-                       for f in range(f_lo, f_hi + 1))
-        elif pattern == STRIPE:
-            # first stripe token at or after uj_lo
-            f = uj_lo // S
-            keep = (uj_lo - f * S) < stripe_blocks * blk or (f + 1) * S <= uj_hi
-        elif pattern == TILE3D:
-            fi_lo, fi_hi = ti_lo // S, ti_hi // S
-            fj_lo, fj_hi = uj_lo // S, uj_hi // S
-            keep = (fj_lo <= fi_hi and fj_hi >= fi_lo) or fj_lo < tile_global_frames
-        else:
-            raise ValueError(pattern)
-        if keep:
-            out.append(j)
-    return out
+    j = np.arange(nb, dtype=np.int64)
+    uj_lo = j * blk
+    uj_hi = np.minimum(n, (j + 1) * blk) - 1
+    if pattern == MULTIDIAG:
+        # offsets u - t over the two blocks form the integer interval [lo, hi]
+        lo, hi = uj_lo - ti_hi, uj_hi - ti_lo
+        keep = np.zeros(nb, dtype=bool)
+        for f in range(f_lo, f_hi + 1):
+            keep |= (lo <= f * S + band_w * blk) & (hi >= f * S - band_w * blk)
+    elif pattern == STRIPE:
+        # the first stripe token at or after uj_lo lies in the block
+        f = uj_lo // S
+        keep = ((uj_lo - f * S) < stripe_blocks * blk) | ((f + 1) * S <= uj_hi)
+    elif pattern == TILE3D:
+        fi_lo, fi_hi = ti_lo // S, ti_hi // S
+        fj_lo, fj_hi = uj_lo // S, uj_hi // S
+        keep = ((fj_lo <= fi_hi) & (fj_hi >= fi_lo)) | (fj_lo < tile_global_frames)
+    else:
+        raise ValueError(pattern)
+    return np.nonzero(keep)[0].tolist()
 
 
 def pattern_mask(head_pattern, B: int, H: int, n: int, blk: int, band_w: int, frame_tokens: int,

@@ -1,0 +1,88 @@
+"""Comparators for GPU-vs-oracle parity (test helpers; no method arithmetic).
+
+Tolerances:
+* CSR masks: identical, except kv-blocks whose oracle p lies within 1e-5 of the
+  row's threshold p (the p of the last block the rule keeps).  In mass mode a
+  row whose cumulative mass at the cut, or one block before it, lies within
+  1e-5 of tau is exempt from equality (its block set is still checked for
+  validity: ascending, in range, forced blocks present, size within the cap).
+* O: max |O_gpu - O_ref| <= 2e-2 and rms(O_gpu - O_ref) / rms(O_ref) <= 1e-2.
+* LSE: max |LSE_gpu - LSE_ref| <= 1e-3 where finite; -inf exactly where the
+  oracle's is -inf (empty rows), and O exactly 0 there.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+MASK_BAND = 1e-5
+O_MAX_ABS = 2e-2
+O_REL_RMS = 1e-2
+LSE_ABS = 1e-3
+
+
+def csr_rows(row_ptr, col_idx):
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    col_idx = np.asarray(col_idx)
+    return [col_idx[row_ptr[r]:row_ptr[r + 1]].tolist() for r in range(len(row_ptr) - 1)]
+
+
+def check_csr_valid(row_ptr, col_idx, nb):
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    assert row_ptr[0] == 0 and np.all(np.diff(row_ptr) >= 0)
+    assert row_ptr[-1] == len(col_idx)
+    for cols in csr_rows(row_ptr, col_idx):
+        assert all(0 <= c < nb for c in cols)
+        assert all(a < b for a, b in zip(cols, cols[1:]))
+
+
+def compare_masks(gpu_rp, gpu_ci, info, nb, mode, mass_tau=0.0, cap=None, forced=None):
+    """Returns (n_rows, n_identical, n_band, n_exempt); asserts the band rule."""
+    check_csr_valid(gpu_rp, gpu_ci, nb)
+    g_rows = csr_rows(gpu_rp, gpu_ci)
+    o_rows = csr_rows(info.row_ptr, info.col_idx)
+    assert len(g_rows) == len(o_rows)
+    probs = info.probs.reshape(-1, nb)
+    ident = band = exempt = 0
+    for r, (g, o) in enumerate(zip(g_rows, o_rows)):
+        if g == o:
+            ident += 1
+            continue
+        if forced is not None:
+            assert set(forced(r)) <= set(g), f"row {r}: forced blocks missing"
+        if mode == 1 and (abs(info.mass_at_cut[r] - mass_tau) <= MASK_BAND or
+                          abs(info.mass_before_cut[r] - mass_tau) <= MASK_BAND):
+            if cap is not None:
+                assert len(g) <= cap + len(set(forced(r)) if forced else 0)
+            exempt += 1
+            continue
+        diff = set(g) ^ set(o)
+        p = probs[r]
+        bad = [j for j in diff if abs(p[j] - info.p_thr[r]) > MASK_BAND]
+        assert not bad, (f"row {r}: blocks {sorted(bad)} differ outside the band "
+                         f"(p={[float(p[j]) for j in sorted(bad)]}, p_thr={info.p_thr[r]})")
+        if mode == 0:
+            assert len(g) == len(o), f"row {r}: top-k size differs"
+        band += 1
+    return len(g_rows), ident, band, exempt
+
+
+def compare_attention(o_gpu, lse_gpu, o_ref, lse_ref, rows_mask=None):
+    """o_*: [..., d] float arrays over the same token set; lse_*: [...]."""
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    lse_gpu = np.asarray(lse_gpu, dtype=np.float64)
+    lse_ref = np.asarray(lse_ref, dtype=np.float64)
+    empty = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse_gpu), empty), "empty-row pattern of LSE differs"
+    assert np.all(o_gpu[empty] == 0.0), "empty rows must give O == 0"
+    err = np.abs(o_gpu - o_ref)
+    max_abs = float(err.max()) if err.size else 0.0
+    denom = float(np.sqrt(np.mean(o_ref ** 2))) if o_ref.size else 0.0
+    rel_rms = float(np.sqrt(np.mean(err ** 2)) / denom) if denom > 0 else float(np.sqrt(np.mean(err ** 2)))
+    fin = ~empty
+    lse_err = float(np.abs(lse_gpu[fin] - lse_ref[fin]).max()) if fin.any() else 0.0
+    assert np.all(np.isfinite(o_gpu)), "non-finite O"
+    assert max_abs <= O_MAX_ABS, f"O max-abs {max_abs:.3e} > {O_MAX_ABS}"
+    assert rel_rms <= O_REL_RMS, f"O rel-RMS {rel_rms:.3e} > {O_REL_RMS}"
+    assert lse_err <= LSE_ABS, f"LSE max-abs {lse_err:.3e} > {LSE_ABS}"
+    return max_abs, rel_rms, lse_err

@@ -1,0 +1,92 @@
+"""The C-ABI library builds, loads and exports every symbol include/bsa.h
+declares; host-side validation rejects bad calls before any launch (these
+paths touch no GPU, so they run on CPU)."""
+import ctypes
+
+import pytest
+
+from block_sparse_attention_asa_b200 import build, bsa
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return bsa.load()
+
+
+def test_exports_every_header_symbol(lib):
+    names = bsa.header_functions()
+    assert {"asa_build_mask", "pattern_mask", "bsa_forward", "bsa_check_device_status",
+            "bsa_status_string", "asa_build_mask_workspace_size", "bsa_forward_workspace_size",
+            "asa_build_mask_max_nnz", "bsa_version"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    for code in range(-7, 1):
+        assert bsa.status_string(code)
+    assert bsa.status_string(12345) == "unknown status"
+
+
+def test_workspace_and_capacity_sizes(lib):
+    # Wan2.1-shaped layer: q̄,k̄ fp32 (2*6144*128*4) + bitmaps (6144*16*4)
+    assert bsa.asa_workspace_size(1, 12, 32760, 128, 64) == 2 * 6144 * 128 * 4 + 6144 * 16 * 4
+    assert bsa.asa_max_nnz(1, 12, 32760, 64, bsa.MODE_MASS, 0, 0.1, 0, 0) == 6144 * 51
+    assert bsa.asa_max_nnz(2, 48, 17776, 64, bsa.MODE_TOPK, 33, 0.0, 0, 4) == 2 * 48 * 278 * 37
+    assert bsa.asa_max_nnz(1, 2, 128, 16, bsa.MODE_TOPK, 3, 0.0, 1, 0) == 16 * 4
+    assert lib.asa_build_mask_workspace_size(1, 1, 100, 96, 16) == 0  # unsupported d
+
+
+def _asa(lib, **kw):
+    a = dict(q=256, k=256, B=1, H=1, N=128, d=64, blk=16, mode=0, topk=1, tau=0.0, ratio=0.0, diag=0,
+             sink=0, scale=0.0, rp=256, ci=256, cap=16, ws=256, wsb=1 << 20)
+    a.update(kw)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return lib.asa_build_mask(vp(a["q"]), vp(a["k"]), a["B"], a["H"], a["N"], a["d"], a["blk"],
+                              a["mode"], a["topk"], a["tau"], a["ratio"], a["diag"], a["sink"],
+                              a["scale"], vp(a["rp"]), vp(a["ci"]), a["cap"], vp(a["ws"]), a["wsb"],
+                              None)
+
+
+def test_asa_validation_rejects_before_launch(lib):
+    assert _asa(lib, q=None) == bsa.ERR_INVALID_ARG
+    assert _asa(lib, B=0) == bsa.ERR_INVALID_ARG
+    assert _asa(lib, d=96) == bsa.ERR_UNSUPPORTED
+    assert _asa(lib, blk=48) == bsa.ERR_UNSUPPORTED
+    assert _asa(lib, q=3) == bsa.ERR_UNSUPPORTED          # misaligned
+    assert _asa(lib, mode=7) == bsa.ERR_INVALID_ARG
+    assert _asa(lib, topk=0) == bsa.ERR_INVALID_ARG
+    assert _asa(lib, mode=1, tau=1.5) == bsa.ERR_INVALID_ARG
+    assert _asa(lib, sink=-1) == bsa.ERR_INVALID_ARG
+    assert _asa(lib, ws=None) == bsa.ERR_WORKSPACE
+    assert _asa(lib, wsb=16) == bsa.ERR_WORKSPACE
+    assert _asa(lib, ws=272) == bsa.ERR_WORKSPACE         # not 256-aligned
+
+
+def test_forward_and_pattern_validation(lib):
+    vp = ctypes.c_void_p
+    args = [vp(16), vp(16), vp(16), 1, 1, 128, 64, 16, vp(16), vp(16), 0.0, vp(16), None, None, 0,
+            None]
+    bad = list(args)
+    bad[0] = None
+    assert lib.bsa_forward(*bad) == bsa.ERR_INVALID_ARG
+    bad = list(args)
+    bad[6] = 80
+    assert lib.bsa_forward(*bad) == bsa.ERR_UNSUPPORTED
+    bad = list(args)
+    bad[7] = 24
+    assert lib.bsa_forward(*bad) == bsa.ERR_UNSUPPORTED
+    bad = list(args)
+    bad[1] = vp(18)
+    assert lib.bsa_forward(*bad) == bsa.ERR_UNSUPPORTED
+    hp = (ctypes.c_int32 * 2)(0, 9)
+    assert lib.pattern_mask(hp, 1, 2, 128, 16, 2, 64, -1, 1, 1, 0, vp(16), vp(16), 8, None,
+                            None) == bsa.ERR_INVALID_ARG
+    hp = (ctypes.c_int32 * 2)(0, 1)
+    assert lib.pattern_mask(hp, 1, 2, 128, 16, 2, 0, -1, 1, 1, 0, vp(16), vp(16), 8, None,
+                            None) == bsa.ERR_INVALID_ARG
+    assert lib.pattern_mask(hp, 1, 2, 128, 16, 2, 64, 2, 1, 1, 0, vp(16), vp(16), 8, None,
+                            None) == bsa.ERR_INVALID_ARG
+    assert lib.pattern_mask(None, 1, 2, 128, 16, 2, 64, -1, 1, 1, 0, vp(16), vp(16), 8, None,
+                            None) == bsa.ERR_INVALID_ARG
