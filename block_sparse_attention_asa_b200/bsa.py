@@ -40,6 +40,9 @@ _SIGNATURES = {
     "asa_build_mask": (_c_int, [_vp, _vp] + [_c_int] * 7 + [_c_float, _c_float, _c_int, _c_int,
                                                              _c_float, _vp, _vp, _c_i64, _vp,
                                                              _c_size, _vp]),
+    "asa_build_mask_noalloc": (_c_int, [_vp, _vp] + [_c_int] * 7 + [_c_float, _c_float, _c_int,
+                                                                     _c_int, _c_float, _vp, _vp,
+                                                                     _c_i64, _vp]),
     "pattern_mask": (_c_int, [_vp] + [_c_int] * 10 + [_vp, _vp, _c_i64, _vp, _vp]),
     "bsa_forward_workspace_size": (_c_size, [_c_int] * 5),
     "bsa_forward": (_c_int, [_vp, _vp, _vp] + [_c_int] * 5 + [_vp, _vp, _c_float, _vp, _vp, _vp,
@@ -163,6 +166,19 @@ def asa_build_mask(q: torch.Tensor, k: torch.Tensor, blk: int, mode: int = MODE_
         nnz = int(row_ptr[-1].item())
         col_idx = col_idx[:nnz]
     return row_ptr, col_idx
+
+
+def asa_build_mask_noalloc_into(q, k, blk, mode, topk, mass_tau, max_keep_ratio, keep_diag,
+                                n_sink_blocks, softmax_scale, row_ptr, col_idx, stream=None):
+    """The ASA mask into preallocated outputs, with the library's own fixed
+    scratch instead of a workspace: for callers that may not allocate device
+    memory.  Asynchronous; concurrent calls on one device must be serialized."""
+    B, H, N, d = _shape(q)
+    rc = load().asa_build_mask_noalloc(_ptr(q), _ptr(k), B, H, N, d, blk, mode, topk, mass_tau,
+                                       max_keep_ratio, keep_diag, n_sink_blocks, softmax_scale,
+                                       _ptr(row_ptr), _ptr(col_idx), col_idx.numel(),
+                                       _stream(stream))
+    _check(rc, "asa_build_mask_noalloc")
 
 
 # ----------------------------------------------------------------------------- patterns

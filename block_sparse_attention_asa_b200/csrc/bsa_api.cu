@@ -374,3 +374,70 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
 }
 
 }  // extern "C"
+
+// ============================================================================
+// asa_build_mask_noalloc: the ASA mask with its scratch in a fixed-size device
+// array that belongs to the library, for callers that cannot allocate device
+// memory (see include/bsa.h).  The array is file-scope and static; host code
+// must not hand its name to a kernel (on the host that name is only a stand-in
+// for the device object), so the device address is looked up with
+// cudaGetSymbolAddress, once per device, on the first call made while that
+// device is current, and that address is what the kernels receive.
+// ============================================================================
+static __device__ __align__(256) unsigned char bsa_asa_noalloc_scratch[BSA_ASA_NOALLOC_MAX_WORKSPACE];
+
+namespace {
+
+constexpr int kNoallocMaxDevices = 64;
+void* g_noalloc_addr[kNoallocMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of this device's copy of the scratch array (nullptr on error).
+void* noalloc_scratch_for_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoallocMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, bsa_asa_noalloc_scratch) != cudaSuccess) return nullptr;
+    g_noalloc_addr[dev] = p;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+
+extern "C" int asa_build_mask_noalloc(const void* q, const void* k, int B, int H, int N, int d,
+                                      int blk, int mode, int topk, float mass_tau,
+                                      float max_keep_ratio, int keep_diag, int n_sink_blocks,
+                                      float softmax_scale, int32_t* row_ptr, int32_t* col_idx,
+                                      int64_t col_capacity, bsa_stream_t stream) {
+  // same argument checks as asa_build_mask, minus the caller's workspace
+  if (!q || !k || !row_ptr || (!col_idx && col_capacity > 0) || col_capacity < 0)
+    return BSA_ERR_INVALID_ARG;
+  int rc = common_shape_checks(B, H, N, blk);
+  if (rc != BSA_OK) return rc;
+  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16)) return BSA_ERR_UNSUPPORTED;
+  if (mode != BSA_MODE_TOPK && mode != BSA_MODE_MASS) return BSA_ERR_INVALID_ARG;
+  if (mode == BSA_MODE_TOPK && topk < 1) return BSA_ERR_INVALID_ARG;
+  if (mode == BSA_MODE_MASS && !(mass_tau > 0.f && mass_tau <= 1.f)) return BSA_ERR_INVALID_ARG;
+  if (!(max_keep_ratio <= 1.0f) || std::isnan(softmax_scale)) return BSA_ERR_INVALID_ARG;
+  if (n_sink_blocks < 0) return BSA_ERR_INVALID_ARG;
+  if ((N + blk - 1) / blk > 65536) return BSA_ERR_UNSUPPORTED;
+  // the scratch this shape needs must fit the fixed array
+  if (asa_layout(B, H, N, d, blk).total > static_cast<size_t>(BSA_ASA_NOALLOC_MAX_WORKSPACE))
+    return BSA_ERR_WORKSPACE;
+  void* ws = noalloc_scratch_for_current_device();
+  if (ws == nullptr) return BSA_ERR_CUDA;
+  // Nothing in the scratch has to start at zero: each call's pooling kernel
+  // writes every pooled row and its selection kernel writes every bitmap word
+  // before anything reads them.
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
+  cudaStream_t s = as_cuda(stream);
+  if (d == 64)
+    return launch_asa<64>(q, k, B, H, N, blk, mode, topk, mass_tau, max_keep_ratio, keep_diag,
+                          n_sink_blocks, scale, row_ptr, col_idx, col_capacity, ws, s);
+  return launch_asa<128>(q, k, B, H, N, blk, mode, topk, mass_tau, max_keep_ratio, keep_diag,
+                         n_sink_blocks, scale, row_ptr, col_idx, col_capacity, ws, s);
+}

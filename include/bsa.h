@@ -97,6 +97,32 @@ int asa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int
                    int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
                    void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
+/* ---- ASA mask without device allocation ---------------------------------
+ * No counterpart on the pages: an interface addition for callers that may not
+ * call cudaMalloc -- e.g. code embedded in a host framework or inference engine
+ * that owns all device memory and forbids allocation while it runs, or a
+ * real-time path where an allocation's implicit synchronization is not
+ * acceptable.  Same arguments and results as asa_build_mask, without the
+ * workspace: the scratch is a fixed array of BSA_ASA_NOALLOC_MAX_WORKSPACE
+ * bytes that the library keeps in the memory of every GPU that loads it, until
+ * the process exits.  Shapes whose asa_build_mask_workspace_size() exceeds it
+ * are rejected with BSA_ERR_WORKSPACE and nothing is launched (16 MiB covers,
+ * e.g., B1 H12 N32760 d128 and B2 H48 N17776 d64 at blk 64).  This function
+ * calls no cudaMalloc, cudaFree or other allocating routine.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture begins.  Every call on a device shares the one array, and
+ * the array keeps the last call's contents (nothing in it needs to start at
+ * zero): calls that may overlap on the GPU -- on different streams, or from
+ * different host threads without ordering -- race on it and must be
+ * serialized by the caller. */
+#define BSA_ASA_NOALLOC_MAX_WORKSPACE (16u << 20)
+int asa_build_mask_noalloc(const void* q, const void* k, int B, int H, int N, int d, int blk,
+                           int mode, int topk, float mass_tau, float max_keep_ratio,
+                           int keep_diag, int n_sink_blocks, float softmax_scale,
+                           int32_t* row_ptr, int32_t* col_idx, int64_t col_capacity,
+                           bsa_stream_t stream);
+
 /* ---- fixed patterns ------------------------------------------------------
  * [SvDiT] 四种注意力模式 (M0 full, M1 skip, M2 diagonal, M3 multi-diagonal,
  * M4 vertical stripe) and [EvDiT] 3.1 (3D attention tile), one pattern per
