@@ -50,6 +50,7 @@ _SIGNATURES = {
     "bsa_check_device_status": (_c_int, [_vp]),
     "bsa_status_string": (ctypes.c_char_p, [_c_int]),
     "bsa_version": (_c_int, []),
+    "bsa_debug_exp2_poly": (_c_int, [_vp, _vp, _c_int, _vp]),
 }
 
 _lib = None
@@ -241,6 +242,15 @@ def bsa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blk: int, row
         col_idx = torch.zeros(1, dtype=torch.int32, device=q.device)
     bsa_forward_into(q, k, v, blk, row_ptr, col_idx, o, lse, softmax_scale, ws, stream)
     return o, lse
+
+
+def debug_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """The attention kernel's FMA-pipe 2^x, evaluated on a CUDA float32 tensor."""
+    _need_cuda(x)
+    y = torch.empty_like(x)
+    _check(load().bsa_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
+           "bsa_debug_exp2_poly")
+    return y
 
 
 def default_scale(d: int) -> float:

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cmath>
 #include <cstring>
+#include <algorithm>
 #include <mutex>
 
 #include "../../include/bsa.h"
@@ -73,6 +74,14 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int rows) 
 }
 
 // ---- forward launch -----------------------------------------------------------
+int sm_count() {
+  static int counts[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (counts[dev] == 0) cudaDeviceGetAttribute(&counts[dev], cudaDevAttrMultiProcessorCount, dev);
+  return counts[dev];
+}
+
 template <int D, int BLK>
 int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
                const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o, float* lse,
@@ -101,14 +110,19 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   p.nb = nb;
   p.nbw = nbw;
   p.nqt = ceil_div(N, 128);
+  p.n_items = B * H * p.nqt;
   p.row_ptr = row_ptr;
   p.col_idx = col_idx;
+  p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.wait_ns = kWaitNs;
-  dim3 grid(p.nqt, B * H);
-  bsa::bsa_fwd_kernel<D, BLK><<<grid, 256, C::SMEM, stream>>>(mq, mk, mv, p);
+  const int sms = sm_count();
+  if (sms <= 0) return BSA_ERR_CUDA;
+  // persistent: one CTA per SM, two item slots per CTA
+  const int grid = std::min(sms, ceil_div(p.n_items, 2));
+  bsa::bsa_fwd_kernel<D, BLK><<<grid, 384, C::SMEM, stream>>>(mq, mk, mv, p);
   return check_launch();
 }
 
@@ -374,6 +388,20 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
 }
 
 }  // extern "C"
+
+namespace {
+__global__ void exp2_poly_kernel(const float* x, float* y, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) y[i] = bsa::exp2_poly(x[i]);
+}
+}  // namespace
+
+extern "C" int bsa_debug_exp2_poly(const float* x, float* y, int n, bsa_stream_t stream) {
+  if (!x || !y || n < 0) return BSA_ERR_INVALID_ARG;
+  if (n == 0) return BSA_OK;
+  exp2_poly_kernel<<<ceil_div(n, 256), 256, 0, as_cuda(stream)>>>(x, y, n);
+  return check_launch();
+}
 
 // ============================================================================
 // asa_build_mask_noalloc: the ASA mask with its scratch in a fixed-size device

@@ -5,27 +5,55 @@
 // online (running max / running sum) softmax is the FlashAttention scheme that
 // both blogs build on.
 //
-// One CTA per (b·h, 128-query tile).  A 128-row tile holds S = 128/blk q-blocks;
-// it walks the ascending UNION of their CSR rows, 128 keys (S kv-blocks) per
-// step, and masks, per row, the kv-blocks its own q-block does not list.  On
-// B200 an M=64 or N=64 tcgen05.mma runs at half the rate of M=N=128, so a
-// 128x128 tile with some masked work beats exact 64-row tiles.
+// Work item = (b·h, 128-query tile).  A tile holds 128/blk q-blocks and walks the
+// ascending UNION of their CSR rows, 128 keys (128/blk gathered kv-blocks) per
+// step, masking per row the kv-blocks its own q-block does not list.  On B200
+// an M=64 or N=64 tcgen05.mma runs at half the rate of M=N=128, so a 128x128
+// step with some masked work beats exact 64-row tiles.
 //
-// Warp roles (256 threads):
-//   warp 0      TMA producer: Q tile once, then per step S gathered K and V
-//               blocks (one box per kv-block and 64-column chunk, 128B swizzle)
-//               into a ring of NST stages.
-//   warp 1      MMA issuer (one thread): S_j = Q K_jᵀ into TMEM (double
-//               buffered), then O += P_{j-1} V_{j-1} with P read from TMEM.
-//   warp 2      TMEM allocation / release.
-//   warps 4-7   softmax: thread = query row = TMEM lane.  Loads S_j, masks,
-//               running max (rescale of O only when the max grows by more than
-//               2^8, else the stale max is kept -- exact, since the final
-//               normalisation uses the same max), exponentials, P (bf16) back
-//               into TMEM over S_j, epilogue O / l and LSE.
+// Persistent CTAs (one per SM), each running TWO independent item slots (A, B)
+// so that one slot's softmax overlaps the other slot's MMAs.  Items are dealt
+// round-robin: slot X of CTA c takes items 2c+X, 2c+X+2G, ... (G = grid size).
 //
-// TMEM columns: S0 [0,128), S1 [128,256), O [256, 256+D).  P_j occupies the
-// first 64 columns of S_{j%2} (two bf16 per 32-bit column).
+// Warp roles (384 threads, three warpgroups):
+//   warp 3      scheduler: per item builds the q-block bitmaps of its CSR rows
+//               and the ascending union list (block id + keep bits) in shared
+//               memory, double-buffered per slot, and prefetches the item's Q
+//               tile into L2.
+//   warp 0      producer (one lane, state in registers): per step takes up to
+//               128/blk list entries, publishes a per-slot step entry (ring
+//               index, first/last, block ids, keep bits) and the gathered K
+//               boxes (TMA, 128B swizzle) into a K ring; the V boxes follow on a
+//               separate front, since V is needed one step later than K.
+//   warps 1, 2  MMA issuers, one thread per slot: S_X = Q_X Kᵀ, then for the
+//               previous step O_X += P_X V with P read from TMEM.  Issuing a
+//               tcgen05.mma costs the issuing thread about as long as the MMA
+//               runs (measured on B200), so each slot has its own issuer.
+//   warp 2      also allocates and releases TMEM.
+//   warps 4-7   softmax + epilogue of slot A;  warps 8-11 the same for slot B.
+//               Thread = query row = TMEM lane.  Raw-score max (3-input max),
+//               packed f32x2 scale/shift and sums, one ex2 per score, lazy
+//               rescale of O (only when the max grows by more than 2^8; exact
+//               because the final normalisation uses the same stale max),
+//               P (bf16) written over S in TMEM.
+//
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
+//
+// Ordering facts the pipeline relies on:
+//   * tcgen05.mma ops issued by one thread execute in order, so S_X may be
+//     overwritten by the QK issued after the PV that read P_X from it;
+//   * the commit that signals S_X(t) ready also covers PV_X(t-1), issued by
+//     the same thread before QK_X(t), so the softmax may rescale O_X without a
+//     further wait;
+//   * ring index s reuses K and V slots two indices later; the PV that frees
+//     the V slot of an earlier step is issued by its slot's thread as soon as
+//     that thread sees its next step (or its END), which needs only K-front
+//     progress, so the producer never waits on work that needs its own next
+//     step;
+//   * a barrier phase is never completed twice before its waiter looks: each
+//     "free" barrier is released only after the front that waits on it has
+//     passed the entry, so every parity wait is unambiguous;
+//   * every wait is bounded (BSA_ERR_TIMEOUT on expiry, then the CTA unwinds).
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -34,10 +62,11 @@
 namespace bsa {
 
 struct FwdParams {
-  int B, H, N, nb, nbw, nqt;      // nqt: number of 128-query tiles
+  int B, H, N, nb, nbw, nqt, n_items;
   const int32_t* row_ptr;
   const int32_t* col_idx;
   float scale_log2;               // softmax scale * log2(e)
+  float scale;                    // softmax scale
   __nv_bfloat16* o;
   float* lse;
   unsigned long long wait_ns;     // bound on every wait
@@ -45,29 +74,132 @@ struct FwdParams {
 
 template <int D, int BLK>
 struct FwdCfg {
-  static constexpr int BM = 128, BN = 128;
-  static constexpr int SLOTS = BN / BLK;            // kv-blocks per step
-  static constexpr int QB = BM / BLK;               // q-blocks per tile
-  static constexpr int NCH = D / 64;                // 64-column swizzle chunks
-  static constexpr int TILE = 128 * D * 2;          // bytes of a 128-row tile
-  static constexpr int CHUNK = 128 * 128;           // bytes of one 128x64 chunk
-  static constexpr int NST = D == 128 ? 2 : 4;      // K/V ring depth
-  static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = TILE;
-  static constexpr int V_OFF = K_OFF + NST * TILE;
-  static constexpr int AUX_OFF = V_OFF + NST * TILE;
-  // aux: barriers (32 x 8 B), tmem base + flags (64 B), stage meta, bitmaps
-  static constexpr int BAR_BYTES = 256;
-  static constexpr int META_OFF = AUX_OFF + BAR_BYTES + 64;
-  static constexpr int META_STRIDE = 16 + 8 * 8;    // nvalid + blocks[8] + keep[8]
-  static constexpr int BM_OFF = META_OFF + NST * META_STRIDE * 4;
-  static constexpr int kMaxBitmapBytes = 16384;
-  static constexpr int SMEM = BM_OFF + kMaxBitmapBytes + 1024;  // + alignment slack
-  static constexpr int O_COL = 256;
+  static constexpr int SLOTS = 128 / BLK;            // kv-blocks per step
+  static constexpr int QB = 128 / BLK;               // q-blocks per tile
+  static constexpr int NCH = D / 64;                 // 64-column swizzle chunks
+  static constexpr int TILE = 128 * D * 2;           // bytes of a 128-row tile
+  static constexpr int CHUNK = 128 * 128;            // bytes of one 128x64 chunk
+  static constexpr int NK = D == 128 ? 2 : 4;        // K ring depth
+  static constexpr int NV = D == 128 ? 2 : 4;        // V ring depth
+  static constexpr int NM = 8;                       // per-slot softmax entries
+  static constexpr int LCAP = 1024;                  // union entries per list segment
+  static constexpr int Q_OFF = 0;                    // Q_A, Q_B
+  static constexpr int K_OFF = 2 * TILE;
+  static constexpr int V_OFF = K_OFF + NK * TILE;
+  static constexpr int AUX_OFF = V_OFF + NV * TILE;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int SMETA_OFF = AUX_OFF + BAR_BYTES;          // 2 x NM step entries
+  static constexpr int SMETA_INTS = 24;
+  static constexpr int VQ_INTS = 8 * 12;                         // producer V-front queue
+  static constexpr int HDR_OFF = SMETA_OFF + (2 * NM * SMETA_INTS + VQ_INTS) * 4;  // 2x2 headers x 8 ints
+  static constexpr int MISC_OFF = HDR_OFF + 2 * 2 * 8 * 4;
+  static constexpr int LIST_OFF = MISC_OFF + 64;                 // 2 slots x 2 bufs x LCAP
+  static constexpr int BM_OFF = LIST_OFF + 2 * 2 * LCAP * 4;     // per-slot bitmaps
+  static constexpr int kMaxBitmapBytes = 4096;                   // per slot
+  static constexpr int SMEM = BM_OFF + 2 * kMaxBitmapBytes + 1024;
+  static constexpr int S_COL = 0, O_COL = 256;
+};
+
+// entry kinds (list headers and per-slot step entries)
+constexpr int kEntryNormal = 0, kEntryEnd = 2;
+
+// Register split (setmaxnreg, per warpgroup): the control warpgroup (producer,
+// MMA, TMEM, scheduler) gives registers to the two softmax warpgroups, which
+// hold a 128-score row each.  The sum must not exceed the launch allocation
+// (384 threads x 168), or the increase would wait forever.
+constexpr int kRegControl = 80, kRegSoftmax = 208;
+static_assert(128 * kRegControl + 256 * kRegSoftmax <= 384 * 168, "register split over budget");
+// list segment header (ints): [0] kind (0 segment, 2 end) [1] bh [2] qt [3] nq
+//                             [4] count [5] first segment [6] last segment
+// list entry: kv-block id | (keep bits over the tile's q-blocks) << 16
+
+// per-slot softmax entry, as ints:
+//  [0] kind (0 normal, 2 end)  [1] first  [2] last  [3] nvalid  [4] bh  [5] qt
+//  [6..13] block ids          [14..21] keep bits (q-blocks of the tile)
+//  [22] ring index of the step (K slot = ring % NK, V slot = ring % NV)
+__device__ __forceinline__ float fast_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// 2^x on the FMA pipe (Cody-Waite reduction, then a minimax polynomial):
+// n = round(x) through the 1.5*2^23 rounding constant, f = x - n in [-1/2, 1/2],
+// 2^f ~ c0 + f(c1 + f(c2 + f c3)) (relative error 7.5e-5, fitted by
+// fit_exp2_poly.py), and 2^n added into the exponent field.  x is clamped to
+// [-126, ...] so the exponent add cannot wrap; below x = -125 the result is a
+// non-negative value under 2^-124 (exact exp2 there is below 3e-38).  Used for a share of the softmax
+// exponentials so that the MUFU pipe is not the bottleneck.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  const float q = fmaf(fmaf(fmaf(0.0551716685295105f, f, 0.2426111251115799f), f,
+                            0.6932609677314758f),
+                       f, 0.9999280571937561f);
+  return __int_as_float(__float_as_int(q) + (__float_as_int(t) << 23));
+}
+
+// Packed two-wide fp32 arithmetic (one instruction for two scores).
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Pairs (of 16 per 32-column chunk) whose exponentials go to the FMA pipe.
+// Measured on B200: the polynomial costs ~9.5 issue cycles per warp-element
+// against MUFU's 8-cycle pipe occupancy, so it only pays once the softmax is
+// MUFU-bound with idle issue slots; off for now.
+constexpr int kPolyPairs = 0;
+
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+
+// Producer state of one item slot (kept in registers: always named, never indexed).
+struct ProdSlot {
+  int sc = 0;         // list segments consumed so far
+  int pos = 0, count = 0;
+  int bh = 0, qt = 0, nq = 0;
+  int tcount = 0;     // softmax entries published
+  int qcount = 0;     // Q tiles loaded
+  bool have = false, lastseg = false, first_tile = false, flushed = false;
+};
+
+// Scheduler state of one item slot.
+struct SchedSlot {
+  int item = 0;       // current item
+  int fills = 0;      // segments published
+  int wpos = 0;       // next bitmap word of the current item
+  int bh = 0, qt = 0, nq = 0;
+  bool mid = false;   // current item has more segments
+  bool done = false;
 };
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = FwdCfg<D, BLK>;
@@ -75,41 +207,54 @@ __global__ void __launch_bounds__(256, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::AUX_OFF);
-  uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;                 // [NST]
-  uint64_t* v_full = bars + 1 + C::NST;        // [NST]
-  uint64_t* kv_empty = bars + 1 + 2 * C::NST;  // [NST]
-  uint64_t* s_full = bars + 1 + 3 * C::NST;    // [2]
-  uint64_t* p_full = s_full + 2;               // [2]
-  uint64_t* o_done = p_full + 2;               // [2]
-  uint64_t* mma_drain = o_done + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::AUX_OFF + C::BAR_BYTES);
-  int* n_union = reinterpret_cast<int*>(tmem_slot + 1);
-  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 2);
-  int* meta = reinterpret_cast<int*>(smem + C::META_OFF);
-  uint32_t* bm = reinterpret_cast<uint32_t*>(smem + C::BM_OFF);
+  uint64_t* k_full = bars;                       // [NK]
+  uint64_t* k_free = k_full + C::NK;             // [NK]
+  uint64_t* v_full = k_free + C::NK;             // [NV]
+  uint64_t* v_free = v_full + C::NV;             // [NV]
+  uint64_t* q_full = v_free + C::NV;             // [2]
+  uint64_t* q_free = q_full + 2;                 // [2]
+  uint64_t* s_full = q_free + 2;                 // [2]
+  uint64_t* p_full = s_full + 2;                 // [2]
+  uint64_t* o_done = p_full + 2;                 // [2]
+  uint64_t* o_free = o_done + 2;                 // [2]
+  uint64_t* m_full = o_free + 2;                 // [2][NM]
+  uint64_t* l_full = m_full + 2 * C::NM;         // [2][2]
+  uint64_t* l_free = l_full + 4;                 // [2][2]
+  uint64_t* mma_drain = l_free + 4;             // [2]
+  int* smeta = reinterpret_cast<int*>(smem + C::SMETA_OFF);
+  int* hdr = reinterpret_cast<int*>(smem + C::HDR_OFF);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  int* abort_flag = reinterpret_cast<int*>(smem + C::MISC_OFF + 4);
+  uint32_t* lists = reinterpret_cast<uint32_t*>(smem + C::LIST_OFF);
+  uint32_t* bm_all = reinterpret_cast<uint32_t*>(smem + C::BM_OFF);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x, bh = blockIdx.y;
-  const int qb0 = qt * C::QB;                         // first q-block of the tile
-  const int nqb = min(C::QB, p.nb - qb0);             // q-blocks present
   const int nbw = p.nbw;
 
-  // ---- setup: barriers, TMEM, per-q-block bitmaps of the CSR rows, union size
   if (tid == 0) {
-    mbar_init(q_full, 1);
-    for (int s = 0; s < C::NST; ++s) {
+    for (int s = 0; s < C::NK; ++s) {
       mbar_init(&k_full[s], 1);
+      mbar_init(&k_free[s], 1);
+    }
+    for (int s = 0; s < C::NV; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&v_free[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
-      mbar_init(&o_done[b], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_free[x], 1);
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], 128);
+      mbar_init(&o_done[x], 1);
+      mbar_init(&o_free[x], 128);
+      for (int s = 0; s < C::NM; ++s) mbar_init(&m_full[x * C::NM + s], 1);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&l_full[x * 2 + b], 1);
+        mbar_init(&l_free[x * 2 + b], 1);
+      }
     }
-    mbar_init(mma_drain, 1);
-    *n_union = 0;
+    mbar_init(&mma_drain[0], 1);
+    mbar_init(&mma_drain[1], 1);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -120,290 +265,542 @@ __global__ void __launch_bounds__(256, 1)
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
-  for (int e = tid; e < C::QB * nbw; e += 256) bm[e] = 0u;
-  __syncthreads();
-  for (int qq = warp; qq < nqb; qq += 8) {
-    const long long r = (long long)bh * p.nb + qb0 + qq;
-    const int e0 = p.row_ptr[r], e1 = p.row_ptr[r + 1];
-    for (int e = e0 + lane; e < e1; e += 32) {
-      const int c = p.col_idx[e];
-      if (c >= 0 && c < p.nb)
-        atomicOr(&bm[qq * nbw + (c >> 5)], 1u << (c & 31));
-      else
-        record_error(BSA_ERR_CSR);
-    }
-  }
-  __syncthreads();
-  {
-    int cnt = 0;
-    for (int w = tid; w < nbw; w += 256) {
-      uint32_t u = 0;
-      for (int qq = 0; qq < nqb; ++qq) u |= bm[qq * nbw + w];
-      cnt += __popc(u);
-    }
-    cnt = warp_sum(cnt);
-    if (lane == 0 && cnt) atomicAdd(n_union, cnt);
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int ntiles = (*n_union + C::SLOTS - 1) / C::SLOTS;
 
-  if (warp == 0) {
-    // ================================================================ producer
-    if (lane == 0 && ntiles > 0) {
-      const int row0 = qt * 128;
-      mbar_arrive_expect_tx(q_full, C::TILE);
-#pragma unroll
-      for (int c = 0; c < C::NCH; ++c)
-        tma_load_3d(smem + C::Q_OFF + c * C::CHUNK, &tm_q, q_full, c * 64, row0, bh);
-      int w = 0, issued = 0;
-      uint32_t word = 0;
-      for (int qq = 0; qq < nqb; ++qq) word |= bm[qq * nbw];
-      for (int j = 0; j < ntiles && !*(volatile int*)abort_flag; ++j) {
-        const int st = j % C::NST;
-        if (j >= C::NST && !mbar_wait(&kv_empty[st], ((j / C::NST) - 1) & 1, p.wait_ns)) {
-          record_error(BSA_ERR_TIMEOUT);
-          *(volatile int*)abort_flag = 1;
-          break;
-        }
-        int* mt = meta + st * C::META_STRIDE;
-        int nvalid = 0, first = 0;
-#pragma unroll
-        for (int s = 0; s < C::SLOTS; ++s) {
-          while (word == 0 && w + 1 < nbw) {
-            ++w;
-            for (int qq = 0; qq < nqb; ++qq) word |= bm[qq * nbw + w];
-          }
-          int blkid = -1;
-          if (word) {
-            const int bit = __ffs(word) - 1;
-            word &= word - 1;
-            blkid = w * 32 + bit;
-          }
-          if (s == 0) first = blkid;
-          int keep = 0;
-          if (blkid >= 0) {
-            ++nvalid;
-            for (int qq = 0; qq < nqb; ++qq)
-              keep |= ((bm[qq * nbw + (blkid >> 5)] >> (blkid & 31)) & 1u) << qq;
-          }
-          mt[1 + s] = blkid >= 0 ? blkid : first;  // unused slots reload a valid block
-          mt[9 + s] = keep;
-        }
-        mt[0] = nvalid;
-        mbar_arrive_expect_tx(&k_full[st], C::TILE);
-#pragma unroll
-        for (int s = 0; s < C::SLOTS; ++s)
-#pragma unroll
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(smem + C::K_OFF + st * C::TILE + c * C::CHUNK + s * BLK * 128, &tm_k,
-                        &k_full[st], c * 64, mt[1 + s] * BLK, bh);
-        mbar_arrive_expect_tx(&v_full[st], C::TILE);
-#pragma unroll
-        for (int s = 0; s < C::SLOTS; ++s)
-#pragma unroll
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(smem + C::V_OFF + st * C::TILE + c * C::CHUNK + s * BLK * 128, &tm_v,
-                        &v_full[st], c * 64, mt[1 + s] * BLK, bh);
-        issued = j + 1;
+  if (warp == 3) {
+    regs_dec<kRegControl>();
+    // ================================================================ scheduler
+    // Per slot: next item (round-robin over the grid), its q-block bitmaps,
+    // then the ascending union list in segments of at most LCAP entries.
+    SchedSlot S0, S1;
+    S0.item = 2 * blockIdx.x;
+    S1.item = 2 * blockIdx.x + 1;
+    uint64_t t_last = global_ns();
+    auto publish = [&](SchedSlot& st, int X) -> bool {
+      // returns true if a segment (or the end marker) was published
+      const int b = st.fills & 1;
+      if (st.fills >= 2) {
+        // one lane polls, the warp follows its answer
+        bool ready = lane == 0 && mbar_try_wait(&l_free[X * 2 + b], ((st.fills >> 1) - 1) & 1);
+        if (!__shfl_sync(0xffffffffu, ready, 0)) return false;
       }
-      // drain: the loads of the last NST issued steps (and Q) must land before exit
-      mbar_wait(q_full, 0, p.wait_ns);
-      for (int t = issued > C::NST ? issued - C::NST : 0; t < issued; ++t) {
-        const int st = t % C::NST;
-        mbar_wait(&k_full[st], (t / C::NST) & 1, p.wait_ns);
-        mbar_wait(&v_full[st], (t / C::NST) & 1, p.wait_ns);
+      int* h = hdr + (X * 2 + b) * 8;
+      uint32_t* list = lists + (X * 2 + b) * C::LCAP;
+      uint32_t* bm = bm_all + X * (C::kMaxBitmapBytes / 4);
+      bool first_seg = false;
+      while (!st.mid) {
+        if (st.item >= p.n_items) {
+          if (lane == 0) {
+            h[0] = kEntryEnd;
+            mbar_arrive(&l_full[X * 2 + b]);
+          }
+          __syncwarp();
+          st.done = true;
+          ++st.fills;
+          return true;
+        }
+        st.bh = st.item / p.nqt;
+        st.qt = st.item % p.nqt;
+        const int qb0 = st.qt * C::QB;
+        st.nq = min(C::QB, p.nb - qb0);
+        for (int e = lane; e < C::QB * nbw; e += 32) bm[e] = 0u;
+        __syncwarp();
+        for (int qq = 0; qq < st.nq; ++qq) {
+          const long long r = (long long)st.bh * p.nb + qb0 + qq;
+          const int e0 = p.row_ptr[r], e1 = p.row_ptr[r + 1];
+          for (int e = e0 + lane; e < e1; e += 32) {
+            const int c = p.col_idx[e];
+            if (c >= 0 && c < p.nb)
+              atomicOr(&bm[qq * nbw + (c >> 5)], 1u << (c & 31));
+            else
+              record_error(BSA_ERR_CSR);
+          }
+        }
+        __syncwarp();
+        int cnt = 0;
+        for (int wd = lane; wd < nbw; wd += 32) {
+          uint32_t u = 0;
+          for (int qq = 0; qq < st.nq; ++qq) u |= bm[qq * nbw + wd];
+          cnt += __popc(u);
+        }
+        cnt = warp_sum(cnt);
+        st.item += 2 * (int)gridDim.x;
+        if (cnt == 0) {
+          // no row of this tile lists anything: O = 0, LSE = -inf
+          for (int r = 0; r < 128; ++r) {
+            const int token = st.qt * 128 + r;
+            if (token >= p.N) break;
+            uint4* dst = reinterpret_cast<uint4*>(p.o + ((long long)st.bh * p.N + token) * D);
+            for (int c = lane; c < D / 8; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+            if (lane == 0 && p.lse) p.lse[(long long)st.bh * p.N + token] = -INFINITY;
+          }
+          continue;
+        }
+        if (lane == 0)
+          for (int c = 0; c < C::NCH; ++c) tma_prefetch_l2_3d(&tm_q, c * 64, st.qt * 128, st.bh);
+        st.mid = true;
+        st.wpos = 0;
+        first_seg = true;
+      }
+      // fill the segment from the union, 32 bitmap words per round
+      int n = 0;
+      while (st.wpos < nbw) {
+        const int wd = st.wpos + lane;
+        uint32_t u = 0;
+        if (wd < nbw)
+          for (int qq = 0; qq < st.nq; ++qq) u |= bm[qq * nbw + wd];
+        const int c = __popc(u);
+        const int incl = warp_incl_scan(c);
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (n + total > C::LCAP) break;  // next segment (a round never exceeds LCAP)
+        int at = n + incl - c;
+        while (u) {
+          const int bit = __ffs(u) - 1;
+          u &= u - 1;
+          const int blk = wd * 32 + bit;
+          uint32_t keep = 0;
+          for (int qq = 0; qq < st.nq; ++qq) keep |= ((bm[qq * nbw + wd] >> bit) & 1u) << qq;
+          list[at++] = static_cast<uint32_t>(blk) | (keep << 16);
+        }
+        n += total;
+        st.wpos += 32;
+      }
+      const bool last_seg = st.wpos >= nbw;
+      __syncwarp();
+      if (lane == 0) {
+        h[0] = 0;
+        h[1] = st.bh;
+        h[2] = st.qt;
+        h[3] = st.nq;
+        h[4] = n;
+        h[5] = first_seg;
+        h[6] = last_seg;
+        mbar_arrive(&l_full[X * 2 + b]);
+      }
+      __syncwarp();
+      st.mid = !last_seg;
+      ++st.fills;
+      return true;
+    };
+    while (!(S0.done && S1.done)) {
+      if (__any_sync(0xffffffffu, *(volatile int*)abort_flag != 0)) break;
+      bool prog = false;
+      if (!S0.done) prog |= publish(S0, 0);
+      if (!S1.done) prog |= publish(S1, 1);
+      if (prog) {
+        t_last = global_ns();
+      } else if (global_ns() - t_last > p.wait_ns) {
+        if (lane == 0) record_error(BSA_ERR_TIMEOUT);
+        *(volatile int*)abort_flag = 1;
+        break;
       }
     }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ================================================================ MMA issuer
-    if (lane == 0 && ntiles > 0) {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t q_base = smem_u32(smem + C::Q_OFF);
-      bool ok = mbar_wait(q_full, 0, p.wait_ns);
-      tc_fence_after();
-      auto issue_pv = [&](int jj) -> bool {
-        const int sb = jj & 1, st = jj % C::NST;
-        if (!mbar_wait(&p_full[sb], (jj >> 1) & 1, p.wait_ns)) return false;
-        if (!mbar_wait(&v_full[st], (jj / C::NST) & 1, p.wait_ns)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(smem + C::V_OFF + st * C::TILE);
+  } else if (warp == 0) {
+    regs_dec<kRegControl>();
+    // ================================================================ producer
+    // Two fronts over the ring: the K front publishes entry sk (ring and
+    // softmax entries, K boxes) once K slot sk % NK is free; the V front loads
+    // the V boxes of entry sv < sk once V slot sv % NV is free.  V is needed one
+    // entry later than K, so a PV still running never holds back the next K.
+    if (lane == 0) {
+      ProdSlot P0, P1;
+      int sk = 0, sv = 0;  // next ring index for K / for V
+      int last = 1;        // slot of the previous ring entry
+      bool ok = true, k_done = false;
+      int* vq = smeta + 2 * C::NM * C::SMETA_INTS;   // V-front queue: 8 entries x 12 ints
+      // One K-front entry for slot X.  Returns false on a wait that gave up.
+      bool used_ring = false;
+      auto k_step = [&](ProdSlot& P, int X) -> bool {
+        used_ring = false;
+        int* vqe = vq + (sk & 7) * 12;
+        if (!P.have || P.pos == P.count) {
+          if (P.have) {
+            mbar_arrive(&l_free[X * 2 + ((P.sc - 1) & 1)]);
+            P.have = false;
+          }
+          const int b = P.sc & 1;
+          if (!mbar_wait(&l_full[X * 2 + b], (P.sc >> 1) & 1, p.wait_ns)) return false;
+          const int* h = hdr + (X * 2 + b) * 8;
+          ++P.sc;
+          if (h[0] == kEntryEnd) {
+            // slot finished: END entry for its softmax and MMA threads (no ring slot)
+            int* sm = smeta + (X * C::NM + P.tcount % C::NM) * C::SMETA_INTS;
+            sm[0] = kEntryEnd;
+            mbar_arrive(&m_full[X * C::NM + P.tcount % C::NM]);
+            P.flushed = true;
+            return true;
+          }
+          P.have = true;
+          P.pos = 0;
+          P.count = h[4];
+          P.lastseg = h[6] != 0;
+          if (h[5]) {
+            P.bh = h[1];
+            P.qt = h[2];
+            P.nq = h[3];
+            P.first_tile = true;
+            // Q tile (after the previous item's last QK on this slot)
+            if (P.qcount > 0 && !mbar_wait(&q_free[X], (P.qcount - 1) & 1, p.wait_ns)) return false;
+            mbar_arrive_expect_tx(&q_full[X], C::TILE);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t db = smem_desc(v_base + kk * 2048, C::CHUNK, 1024);
-          mma_ts(tmem + C::O_COL, tmem + sb * 128 + kk * 8, db, idesc_pv, (jj > 0 || kk > 0));
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_3d(smem + C::Q_OFF + X * C::TILE + c * C::CHUNK, &tm_q, &q_full[X], c * 64,
+                          P.qt * 128, P.bh);
+            ++P.qcount;
+          }
         }
-        mma_commit(&kv_empty[st]);
-        mma_commit(&o_done[sb]);
+        const uint32_t* list = lists + (X * 2 + ((P.sc - 1) & 1)) * C::LCAP;
+        int* sm = smeta + (X * C::NM + P.tcount % C::NM) * C::SMETA_INTS;
+        const int nvalid = min(C::SLOTS, P.count - P.pos);
+        const uint32_t e0 = list[P.pos];
+#pragma unroll
+        for (int sl = 0; sl < C::SLOTS; ++sl) {
+          const uint32_t e = sl < nvalid ? list[P.pos + sl] : e0;   // unused: reload a listed block
+          const int blk = static_cast<int>(e & 0xFFFFu);
+          sm[6 + sl] = blk;
+          sm[14 + sl] = sl < nvalid ? static_cast<int>(e >> 16) : 0;
+          vqe[2 + sl] = blk;
+        }
+        vqe[0] = kEntryNormal;
+        vqe[1] = P.bh;
+        P.pos += nvalid;
+        const int first = P.first_tile ? 1 : 0;
+        const int lastt = (P.lastseg && P.pos == P.count) ? 1 : 0;
+        P.first_tile = false;
+        sm[0] = kEntryNormal;
+        sm[1] = first;
+        sm[2] = lastt;
+        sm[3] = nvalid;
+        sm[4] = P.bh;
+        sm[5] = P.qt;
+        sm[22] = sk;   // ring index: K slot sk % NK, V slot sk % NV
+        mbar_arrive(&m_full[X * C::NM + P.tcount % C::NM]);
+        used_ring = true;
+        ++P.tcount;
+        const int ks = sk % C::NK;
+        mbar_arrive_expect_tx(&k_full[ks], C::TILE);
+#pragma unroll
+        for (int sl = 0; sl < C::SLOTS; ++sl)
+#pragma unroll
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(smem + C::K_OFF + ks * C::TILE + c * C::CHUNK + sl * BLK * 128, &tm_k,
+                        &k_full[ks], c * 64, vqe[2 + sl] * BLK, P.bh);
         return true;
       };
-      for (int j = 0; ok && j < ntiles; ++j) {
-        const int st = j % C::NST, sb = j & 1;
-        if (!mbar_wait(&k_full[st], (j / C::NST) & 1, p.wait_ns)) {
+      uint64_t t_last = global_ns();
+      while (ok) {
+        if (*(volatile int*)abort_flag) break;
+        bool prog = false;
+        // ---- K front
+        if (!k_done && (sk < C::NK || mbar_try_wait(&k_free[sk % C::NK], ((sk / C::NK) - 1) & 1))) {
+          int X = last ^ 1;
+          const bool f0 = P0.flushed, f1 = P1.flushed;
+          if ((X == 0 && f0) || (X == 1 && f1)) X ^= 1;
+          if (f0 && f1) {
+            k_done = true;
+          } else {
+            ok = (X == 0) ? k_step(P0, 0) : k_step(P1, 1);
+            if (!ok) break;
+            last = X;
+            if (used_ring) ++sk;
+          }
+          prog = true;
+        }
+        // ---- V front
+        while (sv < sk && (sv < C::NV || mbar_try_wait(&v_free[sv % C::NV], ((sv / C::NV) - 1) & 1))) {
+          const int* vqe = vq + (sv & 7) * 12;
+          const int vs = sv % C::NV;
+          mbar_arrive_expect_tx(&v_full[vs], C::TILE);
+#pragma unroll
+          for (int sl = 0; sl < C::SLOTS; ++sl)
+#pragma unroll
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_3d(smem + C::V_OFF + vs * C::TILE + c * C::CHUNK + sl * BLK * 128, &tm_v,
+                          &v_full[vs], c * 64, vqe[2 + sl] * BLK, vqe[1]);
+          ++sv;
+          prog = true;
+        }
+        if (k_done && sv == sk) break;
+        if (prog) {
+          t_last = global_ns();
+        } else if (global_ns() - t_last > p.wait_ns) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(smem + C::K_OFF + st * C::TILE);
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          mma_ss(tmem + sb * 128, smem_desc(q_base + off, 16, 1024),
-                 smem_desc(k_base + off, 16, 1024), idesc_qk, kk > 0);
-        }
-        mma_commit(&s_full[sb]);
-        if (j >= 1 && !issue_pv(j - 1)) ok = false;
       }
-      if (ok) ok = issue_pv(ntiles - 1);
       if (!ok) {
         record_error(BSA_ERR_TIMEOUT);
         *(volatile int*)abort_flag = 1;
       }
-      // every MMA this thread issued completes before the CTA releases TMEM
-      mma_commit(mma_drain);
-      mbar_wait(mma_drain, 0, p.wait_ns);
+      // drain: the loads of the last ring entries (and Q) land before exit
+      for (int t = sk > C::NK ? sk - C::NK : 0; t < sk; ++t)
+        mbar_wait(&k_full[t % C::NK], (t / C::NK) & 1, p.wait_ns);
+      for (int t = sv > C::NV ? sv - C::NV : 0; t < sv; ++t)
+        mbar_wait(&v_full[t % C::NV], (t / C::NV) & 1, p.wait_ns);
+      if (P0.qcount > 0) mbar_wait(&q_full[0], (P0.qcount - 1) & 1, p.wait_ns);
+      if (P1.qcount > 0) mbar_wait(&q_full[1], (P1.qcount - 1) & 1, p.wait_ns);
+    }
+    __syncwarp();
+  } else if (warp == 1 || warp == 2) {
+    regs_dec<kRegControl>();
+    // ================================================================ MMA issuers
+    // One thread per slot: issuing a tcgen05.mma costs the issuing thread about
+    // as long as the instruction runs, so a single issuer for both slots would
+    // be the bottleneck.  Within a slot the order is the program order of its
+    // thread: PV_X(t-1) is issued before QK_X(t) (S_X holds P_X), and the
+    // commit that publishes S_X(t) covers PV_X(t-1).
+    if (lane == 0) {
+      const int X = warp - 1;
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      // descriptor bases; per-instruction offsets are compile-time adds to the
+      // address field (addresses stay below 2^18, so the 14-bit field never carries)
+      const uint64_t dq = smem_desc(smem_u32(smem + C::Q_OFF + X * C::TILE), 16, 1024);
+      const uint64_t dk0 = smem_desc(smem_u32(smem + C::K_OFF), 16, 1024);
+      const uint64_t dv0 = smem_desc(smem_u32(smem + C::V_OFF), C::CHUNK, 1024);
+      const uint32_t t_s = tmem + C::S_COL + X * 128, t_o = tmem + C::O_COL + X * 128;
+      int pend = -1, pend_first = 0, pend_last = 0, qc = 0, pc = 0, items = 0;
+      bool ok = true, issued = false;
+      auto issue_pv = [&]() -> bool {
+        const int sp = pend;
+        if (!mbar_wait(&v_full[sp % C::NV], (sp / C::NV) & 1, p.wait_ns)) return false;
+        if (pend_first && items > 0 && !mbar_wait(&o_free[X], (items - 1) & 1, p.wait_ns))
+          return false;
+        if (!mbar_wait(&p_full[X], pc & 1, p.wait_ns)) return false;
+        tc_fence_after();
+        const uint64_t dv = dv0 + static_cast<uint64_t>(((sp % C::NV) * C::TILE) >> 4);
+        const uint32_t acc0 = pend_first ? 0u : 1u;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(t_o, t_s + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                 kk == 0 ? acc0 : 1u);
+        ++pc;
+        mma_commit(&v_free[sp % C::NV]);
+        if (pend_last) {
+          mma_commit(&o_done[X]);
+          ++items;
+        }
+        pend = -1;
+        return true;
+      };
+      for (int t = 0; ok; ++t) {
+        const int mi = X * C::NM + t % C::NM;
+        if (!mbar_wait(&m_full[mi], (t / C::NM) & 1, p.wait_ns)) { ok = false; break; }
+        const int* sm = smeta + mi * C::SMETA_INTS;
+        if (sm[0] == kEntryEnd) break;
+        const int first = sm[1], lastt = sm[2], s = sm[22];
+        const int ks = s % C::NK;
+        if (!mbar_wait(&k_full[ks], (s / C::NK) & 1, p.wait_ns)) { ok = false; break; }
+        if (pend >= 0 && !issue_pv()) { ok = false; break; }
+        if (first) {
+          if (!mbar_wait(&q_full[X], qc & 1, p.wait_ns)) { ok = false; break; }
+          ++qc;
+        }
+        tc_fence_after();
+        const uint64_t dk = dk0 + static_cast<uint64_t>((ks * C::TILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
+          mma_ss(t_s, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        issued = true;
+        mma_commit(&k_free[ks]);
+        if (lastt) mma_commit(&q_free[X]);
+        mma_commit(&s_full[X]);
+        pend = s;
+        pend_first = first;
+        pend_last = lastt;
+      }
+      if (ok && pend >= 0) ok = issue_pv();
+      if (!ok) {
+        record_error(BSA_ERR_TIMEOUT);
+        *(volatile int*)abort_flag = 1;
+      }
+      if (issued) {
+        mma_commit(&mma_drain[X]);
+        mbar_wait(&mma_drain[X], 0, p.wait_ns);
+      }
     }
     __syncwarp();
   } else if (warp >= 4) {
+    regs_inc<kRegSoftmax>();
     // ================================================================ softmax
-    const int wq = warp - 4;                 // TMEM lane quarter
-    const int row = wq * 32 + lane;          // query row in the tile
-    const int qq = row / BLK;                // its q-block in the tile
-    const int token = qt * 128 + row;
+    const int X = (warp >= 8) ? 1 : 0;
+    const int wq = warp & 3;                  // TMEM lane quarter
+    const int row = wq * 32 + lane;           // query row in the tile
+    const int qq = row / BLK;                 // its q-block in the tile
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    float m_run = -INFINITY, l_run = 0.f;
+    const uint32_t s_col = C::S_COL + X * 128, o_col = C::O_COL + X * 128;
+    const float c2 = p.scale_log2;
+    float m_run = -INFINITY;   // running max of raw scores
+    float l_run = 0.f;
+    int items = 0;
     bool ok = true;
-    for (int j = 0; j < ntiles; ++j) {
-      const int sb = j & 1, st = j % C::NST;
-      bool w_ok = mbar_wait(&s_full[sb], (j >> 1) & 1, p.wait_ns) &&
-                  mbar_wait(&k_full[st], (j / C::NST) & 1, p.wait_ns) &&
-                  !*(volatile int*)abort_flag;
-      if (!__all_sync(0xffffffffu, w_ok)) {
-        ok = false;
-        break;
+    for (int t = 0;; ++t) {
+      const int mi = X * C::NM + t % C::NM;
+      bool w_ok = mbar_wait(&m_full[mi], (t / C::NM) & 1, p.wait_ns) && !*(volatile int*)abort_flag;
+      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+      // the entry stays valid until this step's P is published; bh/qt are kept
+      // in registers for the epilogue, which runs after that
+      const int* sm = smeta + mi * C::SMETA_INTS;
+      if (sm[0] == kEntryEnd) break;
+      const int first = sm[1], lastt = sm[2], nvalid = sm[3];
+      const int e_bh = sm[4], e_qt = sm[5];
+      // which slots of the step this row keeps, and the one partial block (the
+      // last, < blk keys) if present; read before S lands
+      uint32_t live_bits = 0;
+      int part_slot = -1, part_keys = BLK;
+#pragma unroll
+      for (int sl = 0; sl < C::SLOTS; ++sl) {
+        if (sl < nvalid && ((sm[14 + sl] >> qq) & 1)) {
+          live_bits |= 1u << sl;
+          const int nk = p.N - sm[6 + sl] * BLK;
+          if (nk < BLK) {
+            part_slot = sl;
+            part_keys = nk;
+          }
+        }
       }
+      const bool live_all = live_bits == (1u << C::SLOTS) - 1u && part_slot < 0;
+      if (first) {
+        m_run = -INFINITY;
+        l_run = 0.f;
+      }
+      w_ok = mbar_wait(&s_full[X], t & 1, p.wait_ns);
+      if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
-      const int* mt = meta + st * C::META_STRIDE;
       float x[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t r[32];
-        tmem_ld32(t_lane + sb * 128 + c * 32, r);
+        tmem_ld32(t_lane + s_col + c * 32, r);
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
       }
       tmem_wait_ld();
-      const int nvalid = mt[0];
-      float tmax = -INFINITY;
+      // masking: slots this row's q-block does not list, unused slots, keys >= N
+      if (!__all_sync(0xffffffffu, live_all)) {
 #pragma unroll
-      for (int s = 0; s < C::SLOTS; ++s) {
-        const bool live = s < nvalid && ((mt[9 + s] >> qq) & 1);
-        const int nkeys = live ? min(BLK, p.N - mt[1 + s] * BLK) : 0;
+        for (int sl = 0; sl < C::SLOTS; ++sl) {
+          const int nk = ((live_bits >> sl) & 1u) ? (sl == part_slot ? part_keys : BLK) : 0;
 #pragma unroll
-        for (int e = 0; e < BLK; ++e) {
-          const int c = s * BLK + e;
-          x[c] = e < nkeys ? x[c] * p.scale_log2 : -INFINITY;
-          tmax = fmaxf(tmax, x[c]);
+          for (int e = 0; e < BLK; ++e)
+            if (e >= nk) x[sl * BLK + e] = -INFINITY;
         }
       }
-      // lazy rescale, decided per warp (tcgen05.ld/st are warp-collective)
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; c += 8) {
+        mx0 = fmax3(mx0, x[c], x[c + 1]);
+        mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
+        mx2 = fmax3(mx2, x[c + 4], x[c + 5]);
+        mx3 = fmax3(mx3, x[c + 6], x[c + 7]);
+      }
+      const float tmax = fmax3(fmax3(mx0, mx1, mx2), mx3, mx3);
+      // lazy rescale (decided per warp: tcgen05.ld/st are warp-collective)
       const float m_new = fmaxf(m_run, tmax);
-      const bool grow = m_new > m_run + 8.0f;
-      const bool any_grow = __any_sync(0xffffffffu, grow);
+      const bool grow = m_run == -INFINITY ? (m_new > -INFINITY) : ((m_new - m_run) * c2 > 8.0f);
       float alpha = 1.0f;
       if (grow) {
-        alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
+        alpha = (m_run == -INFINITY) ? 0.0f : fast_ex2((m_run - m_new) * c2);
         m_run = m_new;
       }
-      if (any_grow && j > 0) {
-        // O holds the sum of PV up to step j-1: wait for it, then scale by alpha
-        w_ok = mbar_wait(&o_done[(j - 1) & 1], ((j - 1) >> 1) & 1, p.wait_ns);
-        if (!__all_sync(0xffffffffu, w_ok)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
+      if (!first && __any_sync(0xffffffffu, grow)) {
+        // O_X holds PV up to the previous step, complete (see header); scale it
+        // before any PV of this step is issued
+        // (16 columns at a time: the 128 scores are still live here)
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_lane + C::O_COL + c * 32, r);
+        for (int c = 0; c < D / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(t_lane + o_col + c * 16, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(t_lane + C::O_COL + c * 32, r);
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st16(t_lane + o_col + c * 16, r);
         }
       }
-      const float m_use = m_run;
-      const bool dead = m_use == -INFINITY;
-      float rsum = 0.f;
+      const float neg_m = m_run == -INFINITY ? 0.f : -m_run * c2;
+      const uint64_t c2x2 = pack2(c2, c2), nmx2 = pack2(neg_m, neg_m);
+      uint64_t ls2a = pack2(0.f, 0.f), ls2b = pack2(0.f, 0.f);
+      const bool emu = kPolyPairs > 0 && __all_sync(0xffffffffu, live_all);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int col = half * 64 + 2 * c;
-          const float p0 = dead ? 0.f : exp2f(x[col] - m_use);
-          const float p1 = dead ? 0.f : exp2f(x[col + 1] - m_use);
-          rsum += p0 + p1;
+        for (int c = 0; c < 16; ++c) {
+          const int col = q4 * 32 + 2 * c;
+          float a0, a1;
+          unpack2(ffma2(pack2(x[col], x[col + 1]), c2x2, nmx2), a0, a1);
+          float p0, p1;
+          if (emu && (c & 15) >= 16 - kPolyPairs) {
+            p0 = exp2_poly(a0);
+            p1 = exp2_poly(a1);
+          } else {
+            p0 = fast_ex2(a0);
+            p1 = fast_ex2(a1);
+          }
+          if (c & 1)
+            ls2b = fadd2(ls2b, pack2(p0, p1));
+          else
+            ls2a = fadd2(ls2a, pack2(p0, p1));
           __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
           pk[c] = *reinterpret_cast<uint32_t*>(&h);
         }
-        tmem_st32(t_lane + sb * 128 + half * 32, pk);
+        tmem_st16(t_lane + s_col + q4 * 16, pk);
       }
+      float la0, la1, lb0, lb1;
+      unpack2(ls2a, la0, la1);
+      unpack2(ls2b, lb0, lb1);
+      float ls[4] = {la0, la1, lb0, lb1};
+      const float rsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
       l_run = l_run * alpha + rsum;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[sb]);
+      mbar_arrive(&p_full[X]);
+      if (lastt) {
+        // ---- epilogue of the item
+        const int bh = e_bh, qt = e_qt;
+        const int token = qt * 128 + row;
+        w_ok = mbar_wait(&o_done[X], items & 1, p.wait_ns);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc_fence_after();
+        const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
+        __nv_bfloat16* orow = p.o + ((long long)bh * p.N + token) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(t_lane + o_col + c * 32, r);
+          tmem_wait_ld();
+          uint32_t packed[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * inv_l,
+                                                     __uint_as_float(r[2 * e + 1]) * inv_l);
+            packed[e] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          if (token < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
+                                  packed[4 * e + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&o_free[X]);
+        if (p.lse != nullptr && token < p.N)
+          p.lse[(long long)bh * p.N + token] =
+              l_run > 0.f ? (m_run * p.scale + logf(l_run)) : -INFINITY;
+        ++items;
+      }
     }
     if (!ok) {
       record_error(BSA_ERR_TIMEOUT);
       *(volatile int*)abort_flag = 1;
     }
-    // ---- epilogue
-    bool have_o = ok && ntiles > 0;
-    if (have_o) {
-      const int jl = ntiles - 1;
-      const bool w_ok = mbar_wait(&o_done[jl & 1], (jl >> 1) & 1, p.wait_ns);
-      if (!__all_sync(0xffffffffu, w_ok)) {
-        record_error(BSA_ERR_TIMEOUT);
-        *(volatile int*)abort_flag = 1;
-        have_o = false;
-      }
-      tc_fence_after();
-    }
-    const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-    __nv_bfloat16* orow = p.o + ((long long)bh * p.N + token) * D;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t r[32];
-      if (have_o) {
-        tmem_ld32(t_lane + C::O_COL + c * 32, r);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = 0u;
-      }
-      uint32_t packed[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * inv_l,
-                                                 __uint_as_float(r[2 * e + 1]) * inv_l);
-        packed[e] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      if (token < p.N) {
-        uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
-      }
-    }
-    if (p.lse != nullptr && token < p.N)
-      p.lse[(long long)bh * p.N + token] =
-          l_run > 0.f ? (m_run * 0.69314718055994531f + logf(l_run)) : -INFINITY;
   }
   tc_fence_before();
   __syncthreads();

@@ -168,6 +168,13 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
  * (BSA_OK if none), and clears it.  bsa_status_string never returns NULL. */
 int bsa_check_device_status(bsa_stream_t stream);
 const char* bsa_status_string(int status);
+/* Diagnostics: y[i] = the attention kernel's FMA-pipe exponential 2^x[i]
+ * (Cody-Waite reduction + degree-3 minimax polynomial, relative error below
+ * 1e-4 for x in [-125, 126]; below that the result is a non-negative value
+ * under 2^-124).  Device
+ * pointers, n floats; asynchronous on `stream`.  For testing the kernel's
+ * arithmetic against the CUDA math library; no counterpart on the pages. */
+int bsa_debug_exp2_poly(const float* x, float* y, int n, bsa_stream_t stream);
 /* Library version as major*10000 + minor*100 + patch. */
 int bsa_version(void);
 

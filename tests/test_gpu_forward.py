@@ -153,3 +153,34 @@ def test_forward_sweep_sampled(cuda_lib, keep, blk):
     rng = np.random.default_rng(5)
     rows = sorted(set(rng.choice(w.H * w.nb, size=96, replace=False).tolist() + [w.nb - 1]))
     _run_and_compare(cuda_lib, q, k, v, blk, rp.cpu().numpy(), ci.cpu().numpy(), rows=rows)
+
+
+def test_exp2_polynomial_against_cuda_exp2(cuda_lib):
+    # the softmax's FMA-pipe exponential vs CUDA's exp2f (torch.exp2 on the GPU)
+    x = torch.cat([torch.linspace(-125.0, 126.0, 2_000_001), torch.linspace(-1, 1, 100_001),
+                   torch.tensor([0.0, -0.5, 0.5, 8.0, -125.0])]).cuda()
+    y = cuda_lib.debug_exp2_poly(x)
+    ref = torch.exp2(x.double())
+    rel = ((y.double() - ref).abs() / ref).max().item()
+    assert rel < 1e-4, rel
+    # below the clamp the result is tiny and non-negative (not exactly zero)
+    z = cuda_lib.debug_exp2_poly(torch.tensor([-125.5, -126.0, -200.0, -1000.0], device="cuda"))
+    assert torch.all(z >= 0) and torch.all(z < 2.0 ** -124)
+
+
+@pytest.mark.parametrize("blk,d", [(128, 128), (64, 128), (16, 64)])
+def test_forward_repeatable_under_load(cuda_lib, blk, d):
+    # many empty rows (items without work), single-slot tails, back-to-back
+    # launches: every launch must finish cleanly and give bit-identical output
+    g = torch.Generator().manual_seed(blk + d)
+    N = 5000
+    q, k, v = (torch.randn(2, 3, N, d, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    nb = -(-N // blk)
+    rp, ci = _random_csr(2 * 3 * nb, nb, seed=blk * 7 + d, p_empty=0.4, p_full=0.05)
+    rpd, cid = torch.as_tensor(rp).cuda(), torch.as_tensor(ci).cuda()
+    o0, l0 = cuda_lib.bsa_forward(q, k, v, blk, rpd, cid)
+    assert cuda_lib.check_device_status() == 0
+    for _ in range(20):
+        o1, l1 = cuda_lib.bsa_forward(q, k, v, blk, rpd, cid)
+        assert cuda_lib.check_device_status() == 0
+        assert torch.equal(o0, o1) and torch.equal(l0, l1)
