@@ -122,7 +122,7 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   if (sms <= 0) return BSA_ERR_CUDA;
   // persistent: one CTA per SM, two item slots per CTA
   const int grid = std::min(sms, ceil_div(p.n_items, 2));
-  bsa::bsa_fwd_kernel<D, BLK><<<grid, 384, C::SMEM, stream>>>(mq, mk, mv, p);
+  bsa::bsa_fwd_kernel<D, BLK><<<grid, bsa::kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, p);
   return check_launch();
 }
 

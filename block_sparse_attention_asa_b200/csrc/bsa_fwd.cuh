@@ -82,7 +82,9 @@ struct FwdCfg {
   static constexpr int NK = D == 128 ? 2 : 4;        // K ring depth
   static constexpr int NV = D == 128 ? 2 : 4;        // V ring depth
   static constexpr int NM = 8;                       // per-slot softmax entries
-  static constexpr int LCAP = 1024;                  // union entries per list segment
+  static constexpr int LCAP = 512;                   // union entries per list segment
+  static constexpr int RW = LCAP / 32;               // bitmap words per fill round (<= LCAP bits)
+  static_assert(RW >= 1 && RW <= 32, "fill round must fit one warp and one segment");
   static constexpr int Q_OFF = 0;                    // Q_A, Q_B
   static constexpr int K_OFF = 2 * TILE;
   static constexpr int V_OFF = K_OFF + NK * TILE;
@@ -96,19 +98,25 @@ struct FwdCfg {
   static constexpr int LIST_OFF = MISC_OFF + 64;                 // 2 slots x 2 bufs x LCAP
   static constexpr int BM_OFF = LIST_OFF + 2 * 2 * LCAP * 4;     // per-slot bitmaps
   static constexpr int kMaxBitmapBytes = 4096;                   // per slot
-  static constexpr int SMEM = BM_OFF + 2 * kMaxBitmapBytes + 1024;
+  static constexpr int XCH_OFF = BM_OFF + 2 * kMaxBitmapBytes;   // row max / sum exchange
+  static constexpr int XCH_BYTES = (2 * 2 * 2 * 128 + 2 * 2 * 128) * 4;
+  static constexpr int SMEM = XCH_OFF + XCH_BYTES + 1024;
   static constexpr int S_COL = 0, O_COL = 256;
 };
 
 // entry kinds (list headers and per-slot step entries)
 constexpr int kEntryNormal = 0, kEntryEnd = 2;
 
+// 20 warps: 4 control warps, then 8 softmax warps per slot (a row's 128 keys
+// split over two warps that share the row's TMEM lane).
+constexpr int kFwdThreads = 640;
 // Register split (setmaxnreg, per warpgroup): the control warpgroup (producer,
-// MMA, TMEM, scheduler) gives registers to the two softmax warpgroups, which
-// hold a 128-score row each.  The sum must not exceed the launch allocation
-// (384 threads x 168), or the increase would wait forever.
-constexpr int kRegControl = 80, kRegSoftmax = 208;
-static_assert(128 * kRegControl + 256 * kRegSoftmax <= 384 * 168, "register split over budget");
+// MMA issuers, scheduler) gives registers to the four softmax warpgroups.  The
+// sum must not exceed the launch allocation (640 threads x 96), or the
+// increase would wait forever.
+constexpr int kRegControl = 72, kRegSoftmax = 96;
+static_assert(128 * kRegControl + 512 * kRegSoftmax <= kFwdThreads * 96, "register split over budget");
+
 // list segment header (ints): [0] kind (0 segment, 2 end) [1] bh [2] qt [3] nq
 //                             [4] count [5] first segment [6] last segment
 // list entry: kv-block id | (keep bits over the tile's q-blocks) << 16
@@ -194,12 +202,13 @@ struct SchedSlot {
   int fills = 0;      // segments published
   int wpos = 0;       // next bitmap word of the current item
   int bh = 0, qt = 0, nq = 0;
+  int total = 0, emitted = 0;   // union size of the current item, entries published
   bool mid = false;   // current item has more segments
   bool done = false;
 };
 
 template <int D, int BLK>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using C = FwdCfg<D, BLK>;
@@ -221,6 +230,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* l_full = m_full + 2 * C::NM;         // [2][2]
   uint64_t* l_free = l_full + 4;                 // [2][2]
   uint64_t* mma_drain = l_free + 4;             // [2]
+  uint64_t* pair_bar = mma_drain + 2;            // [2 slots][4 lane quarters]
   int* smeta = reinterpret_cast<int*>(smem + C::SMETA_OFF);
   int* hdr = reinterpret_cast<int*>(smem + C::HDR_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
@@ -244,9 +254,9 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&q_full[x], 1);
       mbar_init(&q_free[x], 1);
       mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 128);
+      mbar_init(&p_full[x], 256);
       mbar_init(&o_done[x], 1);
-      mbar_init(&o_free[x], 128);
+      mbar_init(&o_free[x], 256);
       for (int s = 0; s < C::NM; ++s) mbar_init(&m_full[x * C::NM + s], 1);
       for (int b = 0; b < 2; ++b) {
         mbar_init(&l_full[x * 2 + b], 1);
@@ -255,6 +265,7 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(&mma_drain[0], 1);
     mbar_init(&mma_drain[1], 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 64);
     *abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
@@ -343,19 +354,23 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < C::NCH; ++c) tma_prefetch_l2_3d(&tm_q, c * 64, st.qt * 128, st.bh);
         st.mid = true;
         st.wpos = 0;
+        st.total = cnt;
+        st.emitted = 0;
         first_seg = true;
       }
-      // fill the segment from the union, 32 bitmap words per round
+      // fill the segment from the union, RW bitmap words per round; a round
+      // holds at most RW * 32 = LCAP blocks, so an empty segment always takes
+      // at least one round
       int n = 0;
       while (st.wpos < nbw) {
         const int wd = st.wpos + lane;
         uint32_t u = 0;
-        if (wd < nbw)
+        if (lane < C::RW && wd < nbw)
           for (int qq = 0; qq < st.nq; ++qq) u |= bm[qq * nbw + wd];
         const int c = __popc(u);
         const int incl = warp_incl_scan(c);
         const int total = __shfl_sync(0xffffffffu, incl, 31);
-        if (n + total > C::LCAP) break;  // next segment (a round never exceeds LCAP)
+        if (n + total > C::LCAP) break;  // rest goes to the next segment
         int at = n + incl - c;
         while (u) {
           const int bit = __ffs(u) - 1;
@@ -366,9 +381,10 @@ __global__ void __launch_bounds__(384, 1)
           list[at++] = static_cast<uint32_t>(blk) | (keep << 16);
         }
         n += total;
-        st.wpos += 32;
+        st.wpos += C::RW;
       }
-      const bool last_seg = st.wpos >= nbw;
+      st.emitted += n;
+      const bool last_seg = st.emitted >= st.total;   // never an empty tail segment
       __syncwarp();
       if (lane == 0) {
         h[0] = 0;
@@ -437,6 +453,7 @@ __global__ void __launch_bounds__(384, 1)
           P.pos = 0;
           P.count = h[4];
           P.lastseg = h[6] != 0;
+          if (P.count == 0) return false;   // never published; refuse to spin on it
           if (h[5]) {
             P.bh = h[1];
             P.qt = h[2];
@@ -628,15 +645,32 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp >= 4) {
     regs_inc<kRegSoftmax>();
     // ================================================================ softmax
-    const int X = (warp >= 8) ? 1 : 0;
+    // Warps 4-11: slot A, 12-19: slot B.  Warp q + 4h (q = lane quarter,
+    // h = key half) handles rows 32q..32q+31 and keys [64h, 64h+64) of each
+    // step; the two halves of a row agree on the running max through a
+    // shared-memory slot and a two-warp mbarrier (bounded wait).
+    const int X = (warp - 4) >> 3;
+    const int h = ((warp - 4) >> 2) & 1;
     const int wq = warp & 3;                  // TMEM lane quarter
     const int row = wq * 32 + lane;           // query row in the tile
     const int qq = row / BLK;                 // its q-block in the tile
+    uint64_t* pbar = &pair_bar[X * 4 + wq];   // the two warps of this lane quarter
+    int puse = 0;
+    auto pair_sync = [&]() -> bool {
+      tc_fence_before();
+      mbar_arrive(pbar);
+      const bool r = mbar_wait(pbar, puse & 1, p.wait_ns);
+      ++puse;
+      tc_fence_after();
+      return __all_sync(0xffffffffu, r);
+    };
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t s_col = C::S_COL + X * 128, o_col = C::O_COL + X * 128;
+    float* xmax = reinterpret_cast<float*>(smem + C::XCH_OFF);        // [2][2 slots][2 halves][128]
+    float* xsum = xmax + 2 * 2 * 2 * 128;                             // [2 slots][2 halves][128]
     const float c2 = p.scale_log2;
-    float m_run = -INFINITY;   // running max of raw scores
-    float l_run = 0.f;
+    float m_run = -INFINITY;   // running max of raw scores (same in both halves)
+    float l_run = 0.f;         // this half's running sum
     int items = 0;
     bool ok = true;
     for (int t = 0;; ++t) {
@@ -664,7 +698,12 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      const bool live_all = live_bits == (1u << C::SLOTS) - 1u && part_slot < 0;
+      // slots overlapping this warp's 64 keys
+      constexpr int SPH = C::SLOTS >= 2 ? C::SLOTS / 2 : 1;    // slots per half
+      const int sl0 = C::SLOTS >= 2 ? h * SPH : 0;
+      const uint32_t half_mask = ((1u << SPH) - 1u) << sl0;
+      const bool live_all = (live_bits & half_mask) == half_mask &&
+                            (part_slot < sl0 || part_slot >= sl0 + SPH);
       if (first) {
         m_run = -INFINITY;
         l_run = 0.f;
@@ -672,11 +711,11 @@ __global__ void __launch_bounds__(384, 1)
       w_ok = mbar_wait(&s_full[X], t & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
-      float x[128];
+      float x[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t r[32];
-        tmem_ld32(t_lane + s_col + c * 32, r);
+        tmem_ld32(t_lane + s_col + h * 64 + c * 32, r);
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
       }
@@ -684,22 +723,28 @@ __global__ void __launch_bounds__(384, 1)
       // masking: slots this row's q-block does not list, unused slots, keys >= N
       if (!__all_sync(0xffffffffu, live_all)) {
 #pragma unroll
-        for (int sl = 0; sl < C::SLOTS; ++sl) {
+        for (int c = 0; c < 64; ++c) {
+          const int key = h * 64 + c;             // key index within the step
+          const int sl = key / BLK, e = key % BLK;
           const int nk = ((live_bits >> sl) & 1u) ? (sl == part_slot ? part_keys : BLK) : 0;
-#pragma unroll
-          for (int e = 0; e < BLK; ++e)
-            if (e >= nk) x[sl * BLK + e] = -INFINITY;
+          if (e >= nk) x[c] = -INFINITY;
         }
       }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; c += 8) {
+      for (int c = 0; c < 64; c += 8) {
         mx0 = fmax3(mx0, x[c], x[c + 1]);
         mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
         mx2 = fmax3(mx2, x[c + 4], x[c + 5]);
         mx3 = fmax3(mx3, x[c + 6], x[c + 7]);
       }
-      const float tmax = fmax3(fmax3(mx0, mx1, mx2), mx3, mx3);
+      const float hmax = fmax3(fmax3(mx0, mx1, mx2), mx3, mx3);
+      // agree on the row max with the other half (double-buffered by step
+      // parity); the barrier also orders both halves' S reads before any P write
+      float* xm = xmax + ((t & 1) * 4 + X * 2) * 128;
+      xm[h * 128 + row] = hmax;
+      if (!pair_sync()) { ok = false; break; }
+      const float tmax = fmaxf(hmax, xm[(h ^ 1) * 128 + row]);
       // lazy rescale (decided per warp: tcgen05.ld/st are warp-collective)
       const float m_new = fmaxf(m_run, tmax);
       const bool grow = m_run == -INFINITY ? (m_new > -INFINITY) : ((m_new - m_run) * c2 > 8.0f);
@@ -709,17 +754,16 @@ __global__ void __launch_bounds__(384, 1)
         m_run = m_new;
       }
       if (!first && __any_sync(0xffffffffu, grow)) {
-        // O_X holds PV up to the previous step, complete (see header); scale it
-        // before any PV of this step is issued
-        // (16 columns at a time: the 128 scores are still live here)
-#pragma unroll
-        for (int c = 0; c < D / 16; ++c) {
+        // O_X holds PV up to the previous step, complete (see header); scale
+        // this warp's half of the columns before any PV of this step
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
           uint32_t r[16];
-          tmem_ld16(t_lane + o_col + c * 16, r);
+          tmem_ld16(t_lane + o_col + h * (D / 2) + c * 16, r);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st16(t_lane + o_col + c * 16, r);
+          tmem_st16(t_lane + o_col + h * (D / 2) + c * 16, r);
         }
       }
       const float neg_m = m_run == -INFINITY ? 0.f : -m_run * c2;
@@ -727,11 +771,11 @@ __global__ void __launch_bounds__(384, 1)
       uint64_t ls2a = pack2(0.f, 0.f), ls2b = pack2(0.f, 0.f);
       const bool emu = kPolyPairs > 0 && __all_sync(0xffffffffu, live_all);
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
+      for (int q2 = 0; q2 < 2; ++q2) {
         uint32_t pk[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          const int col = q4 * 32 + 2 * c;
+          const int col = q2 * 32 + 2 * c;
           float a0, a1;
           unpack2(ffma2(pack2(x[col], x[col + 1]), c2x2, nmx2), a0, a1);
           float p0, p1;
@@ -746,40 +790,42 @@ __global__ void __launch_bounds__(384, 1)
             ls2b = fadd2(ls2b, pack2(p0, p1));
           else
             ls2a = fadd2(ls2a, pack2(p0, p1));
-          __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
-          pk[c] = *reinterpret_cast<uint32_t*>(&h);
+          __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+          pk[c] = *reinterpret_cast<uint32_t*>(&hb);
         }
-        tmem_st16(t_lane + s_col + q4 * 16, pk);
+        // P (bf16 pairs) over S: keys 64h + 32 q2 .. +31 -> columns 32h + 16 q2
+        tmem_st16(t_lane + s_col + h * 32 + q2 * 16, pk);
       }
       float la0, la1, lb0, lb1;
       unpack2(ls2a, la0, la1);
       unpack2(ls2b, lb0, lb1);
-      float ls[4] = {la0, la1, lb0, lb1};
-      const float rsum = (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      l_run = l_run * alpha + rsum;
+      l_run = l_run * alpha + ((la0 + la1) + (lb0 + lb1));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[X]);
       if (lastt) {
-        // ---- epilogue of the item
-        const int bh = e_bh, qt = e_qt;
-        const int token = qt * 128 + row;
+        // ---- epilogue of the item: this warp's half of the O columns
+        const int token = e_qt * 128 + row;
         w_ok = mbar_wait(&o_done[X], items & 1, p.wait_ns);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        const float inv_l = l_run > 0.f ? 1.0f / l_run : 0.f;
-        __nv_bfloat16* orow = p.o + ((long long)bh * p.N + token) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        float* xs = xsum + X * 2 * 128;
+        xs[h * 128 + row] = l_run;
+        if (!pair_sync()) { ok = false; break; }
+        const float l_tot = l_run + xs[(h ^ 1) * 128 + row];
+        const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
+        __nv_bfloat16* orow = p.o + ((long long)e_bh * p.N + token) * D + h * (D / 2);
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t r[32];
-          tmem_ld32(t_lane + o_col + c * 32, r);
+          tmem_ld32(t_lane + o_col + h * (D / 2) + c * 32, r);
           tmem_wait_ld();
           uint32_t packed[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * inv_l,
-                                                     __uint_as_float(r[2 * e + 1]) * inv_l);
-            packed[e] = *reinterpret_cast<uint32_t*>(&h);
+            __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * inv_l,
+                                                      __uint_as_float(r[2 * e + 1]) * inv_l);
+            packed[e] = *reinterpret_cast<uint32_t*>(&hb);
           }
           if (token < p.N) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
@@ -791,9 +837,9 @@ __global__ void __launch_bounds__(384, 1)
         }
         tc_fence_before();
         mbar_arrive(&o_free[X]);
-        if (p.lse != nullptr && token < p.N)
-          p.lse[(long long)bh * p.N + token] =
-              l_run > 0.f ? (m_run * p.scale + logf(l_run)) : -INFINITY;
+        if (h == 0 && p.lse != nullptr && token < p.N)
+          p.lse[(long long)e_bh * p.N + token] =
+              l_tot > 0.f ? (m_run * p.scale + logf(l_tot)) : -INFINITY;
         ++items;
       }
     }

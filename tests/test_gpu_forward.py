@@ -184,3 +184,17 @@ def test_forward_repeatable_under_load(cuda_lib, blk, d):
         o1, l1 = cuda_lib.bsa_forward(q, k, v, blk, rpd, cid)
         assert cuda_lib.check_device_status() == 0
         assert torch.equal(o0, o1) and torch.equal(l0, l1)
+
+
+@pytest.mark.parametrize("blk", [64, 16])
+def test_forward_dense_rows_longer_than_a_list_segment(cuda_lib, blk):
+    # every row lists every block: the union of a tile runs over several of the
+    # kernel's list segments (512 blocks each), including an exactly full one
+    N = 64 * 1100 if blk == 64 else 16 * 1024
+    g = torch.Generator().manual_seed(blk)
+    q, k, v = (torch.randn(1, 1, N, 64, generator=g).to(torch.bfloat16) for _ in range(3))
+    nb = -(-N // blk)
+    rp = (np.arange(nb + 1) * nb).astype(np.int32)
+    ci = np.tile(np.arange(nb, dtype=np.int32), nb)
+    rows = [0, 1, nb // 2, nb - 2, nb - 1]
+    _run_and_compare(cuda_lib, q, k, v, blk, rp, ci, rows=rows)
