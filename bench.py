@@ -68,35 +68,51 @@ def block_flops(w: W.Workload, row_ptr: np.ndarray, col_idx: np.ndarray) -> floa
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """nvidia-smi samples of SM clock and throttle reasons.
+
+    The sampler is started, and its first sample awaited, before the timed
+    region; only samples whose host arrival time lies inside the region set by
+    mark_start()/mark_end() are summarised."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 20
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []          # (host time, line)
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            deadline = time.monotonic() + 15.0
+            while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
         except OSError:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def mark_start(self):
+        self.t0 = time.monotonic()
+
+    def mark_end(self):
+        self.t1 = time.monotonic()
 
     def __exit__(self, *a):
         if self.proc is not None:
+            time.sleep(2.0 * self.PERIOD_MS / 1000.0)   # let the last in-region sample arrive
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -106,7 +122,11 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lo = self.t0 if self.t0 is not None else -float("inf")
+        hi = (self.t1 if self.t1 is not None else float("inf")) + self.PERIOD_MS / 1000.0
+        for ts, ln in self.lines:
+            if not (lo <= ts <= hi):
+                continue
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -269,6 +289,7 @@ def run_gpu(args, rank, world, local):
     with ClockSampler(local) as clk:
         t_all0 = torch.cuda.Event(enable_timing=True)
         t_all1 = torch.cuda.Event(enable_timing=True)
+        clk.mark_start()
         t_all0.record(stream)
         for s in range(args.steps):
             ev[s][0].record(stream)
@@ -278,6 +299,7 @@ def run_gpu(args, rank, world, local):
             ev[s][2].record(stream)
         t_all1.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
     barrier(world)
     total_ms = t_all0.elapsed_time(t_all1)
     mask_ms = [e[0].elapsed_time(e[1]) for e in ev]

@@ -8,16 +8,23 @@
 // forced blocks, CSR out.
 //
 // Kernels, in launch order:
-//   asa_pool_kernel    HBM-bound: streams Q and K once (16-byte loads, fp32
-//                      accumulation in a fixed order), writes q̄, k̄ fp32.
-//   asa_select_kernel  per CTA: R q-block rows of one (b, h).  Scores against
-//                      all k̄ (staged through shared memory), softmax, then a
-//                      per-row radix select on the order key
-//                      (p desc, j asc) -> selection bitmap and count.
-//   csr_scan_kernel    counts -> row_ptr.
-//   asa_expand_kernel  bitmaps -> ascending col_idx.
+//   asa_pool_kernel     HBM-bound: streams Q and K once (16-byte loads, fp32
+//                       accumulation in a fixed order), writes q̄ [row][d] and
+//                       k̄ transposed, k̄ᵀ [bh][d][nb padded to 128].
+//   asa_select_kernel   nb <= 1024.  Per CTA, R q-block rows of one (b, h):
+//                       the score tile S = q̄ k̄ᵀ as a register-blocked fp32
+//                       GEMM (k̄ᵀ streamed through shared memory by cp.async,
+//                       double-buffered), then one warp per row with the row's
+//                       probabilities in registers: softmax, and the cut found
+//                       by bisection over the 32-bit order key with warp
+//                       reductions -> selection bitmap and count.
+//   asa_select_generic_kernel   any nb: the same arithmetic with the row kept in
+//                       shared memory and a radix select on the 64-bit key.
+//   csr_scan_kernel     counts -> row_ptr.
+//   asa_expand_kernel   bitmaps -> ascending col_idx.
 #pragma once
 #include "common.cuh"
+#include "ptx.cuh"
 #include <cuda_bf16.h>
 
 namespace bsa {
@@ -28,8 +35,9 @@ namespace bsa {
 template <int D>
 __global__ void __launch_bounds__(256) asa_pool_kernel(const __nv_bfloat16* __restrict__ q,
                                                        const __nv_bfloat16* __restrict__ k,
-                                                       float* __restrict__ pooled, int BH, int N,
-                                                       int blk, int nb) {
+                                                       float* __restrict__ qbar,
+                                                       float* __restrict__ kbarT, int BH, int N,
+                                                       int blk, int nb, int kt_ld) {
   constexpr int LPR = D / 8;          // lanes per row
   constexpr int RPS = 32 / LPR;       // rows per warp step
   const int lane = threadIdx.x & 31;
@@ -64,22 +72,31 @@ __global__ void __launch_bounds__(256) asa_pool_kernel(const __nv_bfloat16* __re
     for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
   if (sub == 0) {
     const float n = static_cast<float>(nrows);
-    float4 a, b;
-    a.x = acc[0] / n; a.y = acc[1] / n; a.z = acc[2] / n; a.w = acc[3] / n;
-    b.x = acc[4] / n; b.y = acc[5] / n; b.z = acc[6] / n; b.w = acc[7] / n;
-    float* dst = pooled + unit * D + col;
-    reinterpret_cast<float4*>(dst)[0] = a;
-    reinterpret_cast<float4*>(dst)[1] = b;
+    if (!is_k) {
+      float4 a, b;
+      a.x = acc[0] / n; a.y = acc[1] / n; a.z = acc[2] / n; a.w = acc[3] / n;
+      b.x = acc[4] / n; b.y = acc[5] / n; b.z = acc[6] / n; b.w = acc[7] / n;
+      float* dst = qbar + u * D + col;
+      reinterpret_cast<float4*>(dst)[0] = a;
+      reinterpret_cast<float4*>(dst)[1] = b;
+    } else {
+      // k̄ᵀ: the CTA's 8 warps pool 8 consecutive blocks, so for each d their
+      // stores fall into one 32-byte sector.
+      float* dst = kbarT + (bh * D + col) * (long long)kt_ld + i;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) dst[(long long)c * kt_ld] = acc[c] / n;
+    }
   }
 }
 
 // ------------------------------------------------------------------ select
 struct SelectParams {
   const float* qbar;      // [BH*nb, D]
-  const float* kbar;      // [BH*nb, D]
+  const float* kbarT;     // [BH, D, kt_ld]: k̄ transposed, rows padded to kt_ld
   uint32_t* bitmaps;      // [BH*nb, nbw]
   int32_t* row_ptr;       // counts go to row_ptr[r+1]
-  int nb, nbw, rows_per_cta, nb_pad;
+  int nb, nbw, rows_per_cta, nb_pad, kt_ld;
+  int dk;                 // asa_select_kernel: k̄ᵀ rows per cp.async stage
   int mode, topk, cap, keep_diag, n_sink;
   float mass_tau, scale;
 };
@@ -227,7 +244,7 @@ __device__ int mass_count(const float* pr, int nb, float tau, int limit, unsigne
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) asa_select_kernel(const SelectParams p) {
+__global__ void __launch_bounds__(256) asa_select_generic_kernel(const SelectParams p) {
   extern __shared__ __align__(16) unsigned char sel_smem[];
   const int R = p.rows_per_cta;
   float* qs = reinterpret_cast<float*>(sel_smem);                  // [R][D]
@@ -241,7 +258,7 @@ __global__ void __launch_bounds__(256) asa_select_kernel(const SelectParams p) {
   const int bh = blockIdx.y, i0 = blockIdx.x * R;
   const int nrow = min(R, p.nb - i0);
   const float* qrow = p.qbar + ((long long)bh * p.nb + i0) * D;
-  const float* kbh = p.kbar + (long long)bh * p.nb * D;
+  const float* kbh = p.kbarT + (long long)bh * D * p.kt_ld;
 
   for (int e = tid; e < nrow * D; e += 256) qs[e] = qrow[e];
   // scores: thread (ty, tx) -> row ty, columns tx + 16*m of the chunk
@@ -250,8 +267,8 @@ __global__ void __launch_bounds__(256) asa_select_kernel(const SelectParams p) {
     __syncthreads();
     const int nj = min(kKChunk, p.nb - jc);
     for (int e = tid; e < nj * D; e += 256) {
-      const int jj = e / D, dd = e % D;
-      kc[jj * (D + 1) + dd] = kbh[(long long)(jc + jj) * D + dd];
+      const int dd = e / nj, jj = e - dd * nj;
+      kc[jj * (D + 1) + dd] = kbh[(long long)dd * p.kt_ld + jc + jj];
     }
     __syncthreads();
     for (int rr = ty; rr < nrow; rr += 16) {
@@ -315,6 +332,265 @@ __global__ void __launch_bounds__(256) asa_select_kernel(const SelectParams p) {
     if (lane == 0) p.row_ptr[r + 1] = cnt;
     __syncwarp();
   }
+}
+
+// ------------------------------------------------------------------ select, registers
+// Order key of the register path: u = ~bits(p).  p >= 0, so ascending u is
+// descending p, and equal u means equal p; ties go to the lower block index.
+// Block j of a row sits in register r = j / 32 of lane j % 32; lanes past nb
+// hold u = ~0u, which decodes to p = +0 and is never kept.
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// Number of blocks of the row with key <= t (row padding counts only at t = ~0u).
+template <int NPL>
+__device__ __forceinline__ int count_le(const unsigned (&u)[NPL], unsigned t) {
+  int c = 0;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) c += u[r] <= t ? 1 : 0;
+  return __reduce_add_sync(0xffffffffu, c);
+}
+
+// Probability mass of the blocks with key <= t (fixed summation order for a given t).
+template <int NPL>
+__device__ __forceinline__ float mass_le(const unsigned (&u)[NPL], unsigned t) {
+  float s = 0.f;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) s += u[r] <= t ? __uint_as_float(~u[r]) : 0.f;
+  return warp_sum_f(s);
+}
+
+// Smallest key t in [lo, hi] with count_le(t) >= m, given count_le(hi) >= m:
+// bisection over the bits below the common prefix of lo and hi.
+template <int NPL>
+__device__ __forceinline__ unsigned kth_by_count(const unsigned (&u)[NPL], int m, unsigned lo,
+                                                 unsigned hi) {
+  if (lo == hi) return lo;
+  const int hb = 31 - __clz(lo ^ hi);
+  unsigned t = lo & ~((2u << hb) - 1u);
+#pragma unroll 1
+  for (int b = hb; b >= 0; --b) {
+    const unsigned bit = 1u << b;
+    if (count_le(u, t | (bit - 1u)) < m) t |= bit;
+  }
+  return t;
+}
+
+// Smallest key t in [lo, hi] with mass_le(t) >= tau, given mass_le(hi) >= tau.
+template <int NPL>
+__device__ __forceinline__ unsigned kth_by_mass(const unsigned (&u)[NPL], float tau, unsigned lo,
+                                                unsigned hi) {
+  if (lo == hi) return lo;
+  const int hb = 31 - __clz(lo ^ hi);
+  unsigned t = lo & ~((2u << hb) - 1u);
+#pragma unroll 1
+  for (int b = hb; b >= 0; --b) {
+    const unsigned bit = 1u << b;
+    if (mass_le(u, t | (bit - 1u)) < tau) t |= bit;
+  }
+  return t;
+}
+
+// Bit r set <=> this lane's block in register r is among the first blocks in
+// key order: every key < T, and the `need` lowest-index blocks with key == T.
+template <int NPL>
+__device__ __forceinline__ unsigned keep_bits(const unsigned (&u)[NPL], int nb, unsigned T,
+                                              int need) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = lanemask_lt();
+  unsigned bits = 0u;
+  int taken = 0;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const bool tie = r * 32 + lane < nb && u[r] == T;
+    const unsigned bal = __ballot_sync(0xffffffffu, tie);
+    const bool k = u[r] < T || (tie && taken + __popc(bal & lt) < need);
+    bits |= (k ? 1u : 0u) << r;
+    taken += __popc(bal);
+  }
+  return bits;
+}
+
+// One warp: softmax of the row's scores, the rule's cut, forced blocks, then
+// the row's bitmap words and count.
+template <int NPL>
+__device__ __forceinline__ void select_row_regs(const float* srow, int i, long long row,
+                                                const SelectParams& p) {
+  const int lane = threadIdx.x & 31;
+  const int nb = p.nb;
+  float v[NPL];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const int j = r * 32 + lane;
+    v[r] = j < nb ? srow[j] : -INFINITY;
+    mx = fmaxf(mx, v[r]);
+  }
+  mx = warp_max(mx);
+  float sum = 0.f;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const float e = r * 32 + lane < nb ? expf(v[r] - mx) : 0.f;
+    v[r] = e;
+    sum += e;
+  }
+  sum = warp_sum_f(sum);
+  const float inv = 1.0f / sum;
+  unsigned u[NPL];
+  unsigned lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    u[r] = 0xFFFFFFFFu;
+    if (r * 32 + lane < nb) {
+      u[r] = ~__float_as_uint(v[r] * inv);
+      lo = min(lo, u[r]);
+      hi = max(hi, u[r]);
+    }
+  }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+
+  const int L = min(p.cap, nb);
+  const int m0 = p.mode == BSA_MODE_TOPK ? min(p.topk, L) : L;
+  unsigned T = kth_by_count(u, m0, lo, hi);
+  int need = m0 - (T == 0u ? 0 : count_le(u, T - 1u));
+  if (p.mode == BSA_MODE_MASS) {
+    // The top L fall short of tau: the cap binds and the cut is L.  Otherwise
+    // the shortest prefix reaching tau ends inside the top L: find its last key.
+    const unsigned kb = keep_bits(u, nb, T, need);
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) s += (kb >> r) & 1u ? __uint_as_float(~u[r]) : 0.f;
+    s = warp_sum_f(s);
+    if (s >= p.mass_tau && mass_le(u, T) >= p.mass_tau) {
+      const unsigned t = kth_by_mass(u, p.mass_tau, lo, T);
+      const int c_lt = t == 0u ? 0 : count_le(u, t - 1u);
+      const float f_lt = t == 0u ? 0.f : mass_le(u, t - 1u);
+      const int n_tie = count_le(u, t) - c_lt;
+      const float pt = __uint_as_float(~t);
+      // ties at the cut are taken one at a time, each adding pt
+      int n = 1;
+      if (pt > 0.f) {
+        const float q = (p.mass_tau - f_lt) / pt;
+        n = q >= static_cast<float>(n_tie) ? n_tie : max(1, static_cast<int>(ceilf(q)));
+      }
+      if (c_lt + n <= L) {
+        T = t;
+        need = n;
+      }
+    }
+  }
+  const unsigned kb = keep_bits(u, nb, T, need);
+  unsigned myword = 0u;
+  int cnt = 0;
+#pragma unroll
+  for (int r = 0; r < NPL; ++r) {
+    const int j = r * 32 + lane;
+    const bool forced = j < nb && ((p.keep_diag && j == i) || j < p.n_sink);
+    const unsigned w = __ballot_sync(0xffffffffu, ((kb >> r) & 1u) || forced);
+    if (lane == r) myword = w;
+    cnt += __popc(w);
+  }
+  if (lane < p.nbw) p.bitmaps[row * p.nbw + lane] = myword;
+  if (lane == 0) p.row_ptr[row + 1] = cnt;
+}
+
+// nb <= 32 * NPL <= 1024.  R = rows_per_cta in {8, 16, 32, 64}, nb_pad =
+// 128 * ncb >= kt_ld with (R / 8) * ncb <= 8: warp w owns the 8 x 128 score tile
+// (rows 8 * (w / ncb) .., columns 128 * (w % ncb) ..), a lane 8 rows x 4
+// columns, so one k̄ᵀ float4 and two broadcast q̄ float4 feed 32 FMAs.
+// Shared memory: qs [D][R] fp32, then region A: two stages of dk k̄ᵀ rows
+// (dk * nb_pad floats each), reused for the [R][nb_pad] scores.
+template <int D, int NPL>
+__global__ void __launch_bounds__(256, NPL == 32 ? 2 : 3) asa_select_kernel(const SelectParams p) {
+  extern __shared__ __align__(16) float sel_f[];
+  const int R = p.rows_per_cta, nb_pad = p.nb_pad, DK = p.dk;
+  float* qs = sel_f;
+  float* ka = sel_f + D * R;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int bh = blockIdx.y, i0 = blockIdx.x * R;
+  const int nrow = min(R, p.nb - i0);
+  const int ncb = nb_pad >> 7;
+  const int rt = warp / ncb, ct = warp - rt * ncb;
+  const bool active = warp < (R >> 3) * ncb && rt * 8 < nrow;
+  const float* kt = p.kbarT + (long long)bh * D * p.kt_ld;
+
+  // stage c: k̄ᵀ rows [c*DK, c*DK+DK) -> buffer c&1 (row stride nb_pad; the
+  // columns past kt_ld are never read back as scores of real blocks)
+  auto stage = [&](int c) {
+    const int ld4 = p.kt_ld >> 2;
+    const float* src = kt + (long long)c * DK * p.kt_ld;
+    float* dst = ka + (c & 1) * DK * nb_pad;
+    for (int rr = warp; rr < DK; rr += kSelWarps)
+      for (int c4 = lane; c4 < ld4; c4 += 32)
+        cp_async16(dst + rr * nb_pad + 4 * c4, src + (long long)rr * p.kt_ld + 4 * c4);
+    cp_async_commit();
+  };
+  stage(0);
+  // q̄ rows -> qs[d][row] (absent rows as zeros)
+  const float* qg = p.qbar + ((long long)bh * p.nb + i0) * D;
+  for (int e = tid; e < R * (D / 4); e += 256) {
+    const int rr = e % R, d4 = e / R;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (rr < nrow) v = __ldg(reinterpret_cast<const float4*>(qg + (long long)rr * D) + d4);
+    qs[(4 * d4 + 0) * R + rr] = v.x;
+    qs[(4 * d4 + 1) * R + rr] = v.y;
+    qs[(4 * d4 + 2) * R + rr] = v.z;
+    qs[(4 * d4 + 3) * R + rr] = v.w;
+  }
+
+  float acc[8][4];
+#pragma unroll
+  for (int a = 0; a < 8; ++a)
+#pragma unroll
+    for (int m = 0; m < 4; ++m) acc[a][m] = 0.f;
+  const int nchunks = D / DK;
+#pragma unroll 1
+  for (int c = 0; c < nchunks; ++c) {
+    if (c + 1 < nchunks) {
+      stage(c + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    if (active) {
+      const float* kb = ka + (c & 1) * DK * nb_pad + ct * 128 + 4 * lane;
+      const float* qb = qs + c * DK * R + rt * 8;
+#pragma unroll 4
+      for (int dd = 0; dd < DK; ++dd) {
+        const float4 kv = *reinterpret_cast<const float4*>(kb + dd * nb_pad);
+        const float4 qa = *reinterpret_cast<const float4*>(qb + dd * R);
+        const float4 qc = *reinterpret_cast<const float4*>(qb + dd * R + 4);
+        const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qc.x, qc.y, qc.z, qc.w};
+        const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+        for (int a = 0; a < 8; ++a)
+#pragma unroll
+          for (int m = 0; m < 4; ++m) acc[a][m] = fmaf(qv[a], kk[m], acc[a][m]);
+      }
+    }
+    __syncthreads();
+  }
+  // scores -> region A (every stage has been consumed)
+  if (active) {
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+      float4 o;
+      o.x = acc[a][0] * p.scale;
+      o.y = acc[a][1] * p.scale;
+      o.z = acc[a][2] * p.scale;
+      o.w = acc[a][3] * p.scale;
+      *reinterpret_cast<float4*>(ka + (rt * 8 + a) * nb_pad + ct * 128 + 4 * lane) = o;
+    }
+  }
+  __syncthreads();
+  for (int rr = warp; rr < nrow; rr += kSelWarps)
+    select_row_regs<NPL>(ka + rr * nb_pad, i0 + rr, (long long)bh * p.nb + i0 + rr, p);
 }
 
 // ------------------------------------------------------------------ expand

@@ -140,20 +140,24 @@ int launch_fwd_blk(int blk, const void* q, const void* k, const void* v, int B, 
 }
 
 // ---- ASA mask sizes -------------------------------------------------------------
+// Workspace: q̄ [rows][d] fp32 | k̄ᵀ [B*H][d][kt_ld] fp32 | bitmaps [rows][nbw] u32,
+// each part starting on a 256-byte boundary.
 struct AsaLayout {
-  long long nb, nbw, rows;
-  size_t pooled_bytes, bitmap_bytes, total;
+  long long nb, nbw, rows, kt_ld;
+  size_t qbar_off, kbar_off, bitmap_off, total;
 };
 
 AsaLayout asa_layout(int B, int H, int N, int d, int blk) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   AsaLayout L;
   L.nb = (N + blk - 1) / blk;
   L.nbw = (L.nb + 31) / 32;
   L.rows = (long long)B * H * L.nb;
-  L.pooled_bytes = (size_t)2 * L.rows * d * sizeof(float);
-  L.bitmap_bytes = (size_t)L.rows * L.nbw * sizeof(uint32_t);
-  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  L.total = up(L.pooled_bytes) + up(L.bitmap_bytes);
+  L.kt_ld = (L.nb + 3) / 4 * 4;   // 16-byte rows for cp.async
+  L.qbar_off = 0;
+  L.kbar_off = up((size_t)L.rows * d * sizeof(float));
+  L.bitmap_off = L.kbar_off + up((size_t)B * H * d * L.kt_ld * sizeof(float));
+  L.total = L.bitmap_off + up((size_t)L.rows * L.nbw * sizeof(uint32_t));
   return L;
 }
 
@@ -164,10 +168,41 @@ int select_cap(int nb, float ratio) {
 }
 
 template <int D>
-size_t select_smem(int R, int nb_pad, int nbw) {
-  (void)nbw;
+size_t select_generic_smem(int R, int nb_pad) {
   return (size_t)R * D * 4 + (size_t)bsa::kKChunk * (D + 1) * 4 + (size_t)R * nb_pad * 4 +
          (size_t)bsa::kSelWarps * 256 * 4 + (size_t)bsa::kSelWarps * 64 * 8;
+}
+
+// Raise a kernel's dynamic shared memory limit once per device.
+template <typename K>
+bool allow_smem(K kernel, int bytes, bool (&done)[64]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  if (dev < 64 && done[dev]) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  if (dev < 64) done[dev] = true;
+  return true;
+}
+
+template <int D, int NPL>
+int launch_select_regs(bsa::SelectParams sp, int BH, cudaStream_t stream) {
+  // R rows per CTA so that the (R/8) x ncb warp tiles fill at most the 8 warps;
+  // dk = k̄ᵀ rows per stage, a power of two with dk * nb_pad <= 8192 floats.
+  const int ncb = (sp.nb + 127) / 128;
+  sp.nb_pad = ncb * 128;
+  sp.rows_per_cta = 8 * (8 / ncb);
+  int dk = D;
+  while (dk * sp.nb_pad > 8192) dk >>= 1;
+  sp.dk = dk;
+  const size_t region_a = std::max((size_t)2 * dk * sp.nb_pad, (size_t)sp.rows_per_cta * sp.nb_pad);
+  const size_t smem = ((size_t)D * sp.rows_per_cta + region_a) * sizeof(float);
+  static bool done[64] = {};
+  if (!allow_smem(bsa::asa_select_kernel<D, NPL>, 112 * 1024, done)) return BSA_ERR_CUDA;
+  dim3 grid(ceil_div(sp.nb, sp.rows_per_cta), BH);
+  bsa::asa_select_kernel<D, NPL><<<grid, 256, smem, stream>>>(sp);
+  return check_launch() ? BSA_ERR_CUDA : BSA_OK;
 }
 
 template <int D>
@@ -177,44 +212,30 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
   const AsaLayout L = asa_layout(B, H, N, D, blk);
   const int nb = static_cast<int>(L.nb), nbw = static_cast<int>(L.nbw);
   const int BH = B * H;
-  float* pooled = static_cast<float*>(ws);
-  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(static_cast<char*>(ws) +
-                                                  ((L.pooled_bytes + 255) & ~(size_t)255));
+  if (BH > 65535) return BSA_ERR_UNSUPPORTED;
+  char* base = static_cast<char*>(ws);
+  float* qbar = reinterpret_cast<float*>(base + L.qbar_off);
+  float* kbarT = reinterpret_cast<float*>(base + L.kbar_off);
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(base + L.bitmap_off);
   // 1. pooling
   {
     const long long units = 2LL * BH * nb;
     bsa::asa_pool_kernel<D><<<ceil_div(units, 8), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), pooled, BH, N,
-        blk, nb);
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar, kbarT,
+        BH, N, blk, nb, static_cast<int>(L.kt_ld));
     if (check_launch()) return BSA_ERR_CUDA;
   }
   // 2. scores + selection
   {
-    const int nb_pad = (nb + 31) / 32 * 32;
-    const size_t budget = 200 * 1024;
-    int R = 16;
-    while (R > 1 && select_smem<D>(R, nb_pad, nbw) > budget) --R;
-    const size_t smem = select_smem<D>(R, nb_pad, nbw);
-    if (smem > budget) return BSA_ERR_UNSUPPORTED;
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-      if (cudaFuncSetAttribute(bsa::asa_select_kernel<D>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024) !=
-          cudaSuccess)
-        return BSA_ERR_CUDA;
-      attr_set[dev] = true;
-    }
     bsa::SelectParams sp;
-    sp.qbar = pooled;
-    sp.kbar = pooled + (size_t)BH * nb * D;
+    sp.qbar = qbar;
+    sp.kbarT = kbarT;
     sp.bitmaps = bitmaps;
     sp.row_ptr = row_ptr;
     sp.nb = nb;
     sp.nbw = nbw;
-    sp.rows_per_cta = R;
-    sp.nb_pad = nb_pad;
+    sp.kt_ld = static_cast<int>(L.kt_ld);
+    sp.dk = 0;
     sp.mode = mode;
     sp.topk = topk;
     sp.cap = select_cap(nb, ratio);
@@ -222,9 +243,27 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
     sp.n_sink = n_sink;
     sp.mass_tau = tau;
     sp.scale = scale;
-    dim3 grid(ceil_div(nb, R), BH);
-    bsa::asa_select_kernel<D><<<grid, 256, smem, stream>>>(sp);
-    if (check_launch()) return BSA_ERR_CUDA;
+    int rc = BSA_OK;
+    if (nb <= 128) rc = launch_select_regs<D, 4>(sp, BH, stream);
+    else if (nb <= 256) rc = launch_select_regs<D, 8>(sp, BH, stream);
+    else if (nb <= 512) rc = launch_select_regs<D, 16>(sp, BH, stream);
+    else if (nb <= 1024) rc = launch_select_regs<D, 32>(sp, BH, stream);
+    else {
+      const int nb_pad = (nb + 31) / 32 * 32;
+      const size_t budget = 200 * 1024;
+      int R = 16;
+      while (R > 1 && select_generic_smem<D>(R, nb_pad) > budget) --R;
+      const size_t smem = select_generic_smem<D>(R, nb_pad);
+      if (smem > budget) return BSA_ERR_UNSUPPORTED;
+      static bool done[64] = {};
+      if (!allow_smem(bsa::asa_select_generic_kernel<D>, 220 * 1024, done)) return BSA_ERR_CUDA;
+      sp.rows_per_cta = R;
+      sp.nb_pad = nb_pad;
+      dim3 grid(ceil_div(nb, R), BH);
+      bsa::asa_select_generic_kernel<D><<<grid, 256, smem, stream>>>(sp);
+      rc = check_launch() ? BSA_ERR_CUDA : BSA_OK;
+    }
+    if (rc != BSA_OK) return rc;
   }
   // 3. counts -> row_ptr
   bsa::csr_scan_kernel<<<1, 1024, 0, stream>>>(row_ptr, static_cast<int>(L.rows));

@@ -104,6 +104,9 @@ ASA_SMALL = [
     (2, 2, 70, 64, 16, 0, 2, 0.0, 0.0, 0, 7),         # sinks cover every block
     (1, 2, 9000, 128, 16, 1, 0, 0.3, 0.05, 0, 1),     # nb 563, ragged
     (1, 1, 20, 64, 64, 0, 1, 0.0, 0.0, 1, 0),         # N < blk
+    (1, 2, 20000, 64, 16, 0, 40, 0.0, 0.0, 1, 1),     # nb 1250: shared-memory select path
+    (1, 1, 20000, 128, 16, 1, 0, 0.6, 0.3, 0, 0),     # nb 1250, mass mode
+    (1, 2, 16384, 64, 16, 1, 0, 0.8, 0.0, 1, 0),      # nb 1024 exactly, uncapped mass
 ]
 
 
