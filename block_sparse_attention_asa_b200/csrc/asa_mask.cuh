@@ -364,19 +364,32 @@ __device__ __forceinline__ float mass_le(const unsigned (&u)[NPL], unsigned t) {
   return warp_sum_f(s);
 }
 
-// Smallest key t in [lo, hi] with count_le(t) >= m, given count_le(hi) >= m:
-// bisection over the bits below the common prefix of lo and hi.
+// The first m blocks in key order (1 <= m <= nb), as (T, need): every key < T
+// and the `need` lowest-index blocks with key == T.  Bisection over the bits
+// below the common prefix of lo and hi (the row's smallest and largest key)
+// for the smallest t with count_le(t) >= m; it stops early at a t with exactly
+// m keys <= t, which then are the answer (T = t + 1, need = 0).
 template <int NPL>
-__device__ __forceinline__ unsigned kth_by_count(const unsigned (&u)[NPL], int m, unsigned lo,
-                                                 unsigned hi) {
-  if (lo == hi) return lo;
+__device__ __forceinline__ unsigned cut_by_count(const unsigned (&u)[NPL], int m, unsigned lo,
+                                                 unsigned hi, int& need) {
+  if (lo == hi) {   // every key equal: the m lowest indices
+    need = m;
+    return lo;
+  }
   const int hb = 31 - __clz(lo ^ hi);
   unsigned t = lo & ~((2u << hb) - 1u);
 #pragma unroll 1
   for (int b = hb; b >= 0; --b) {
     const unsigned bit = 1u << b;
-    if (count_le(u, t | (bit - 1u)) < m) t |= bit;
+    const unsigned cand = t | (bit - 1u);
+    const int c = count_le(u, cand);
+    if (c == m && cand != 0xFFFFFFFFu) {
+      need = 0;
+      return cand + 1u;
+    }
+    if (c < m) t |= bit;
   }
+  need = m - (t == 0u ? 0 : count_le(u, t - 1u));
   return t;
 }
 
@@ -456,8 +469,8 @@ __device__ __forceinline__ void select_row_regs(const float* srow, int i, long l
 
   const int L = min(p.cap, nb);
   const int m0 = p.mode == BSA_MODE_TOPK ? min(p.topk, L) : L;
-  unsigned T = kth_by_count(u, m0, lo, hi);
-  int need = m0 - (T == 0u ? 0 : count_le(u, T - 1u));
+  int need = 0;
+  unsigned T = cut_by_count(u, m0, lo, hi, need);
   if (p.mode == BSA_MODE_MASS) {
     // The top L fall short of tau: the cap binds and the cut is L.  Otherwise
     // the shortest prefix reaching tau ends inside the top L: find its last key.
@@ -466,8 +479,9 @@ __device__ __forceinline__ void select_row_regs(const float* srow, int i, long l
 #pragma unroll
     for (int r = 0; r < NPL; ++r) s += (kb >> r) & 1u ? __uint_as_float(~u[r]) : 0.f;
     s = warp_sum_f(s);
-    if (s >= p.mass_tau && mass_le(u, T) >= p.mass_tau) {
-      const unsigned t = kth_by_mass(u, p.mass_tau, lo, T);
+    const unsigned top = need == 0 ? T - 1u : T;   // largest key among the top L
+    if (s >= p.mass_tau && mass_le(u, top) >= p.mass_tau) {
+      const unsigned t = kth_by_mass(u, p.mass_tau, lo, top);
       const int c_lt = t == 0u ? 0 : count_le(u, t - 1u);
       const float f_lt = t == 0u ? 0.f : mass_le(u, t - 1u);
       const int n_tie = count_le(u, t) - c_lt;
