@@ -252,6 +252,8 @@ def run_gpu(args, rank, world, local):
         ws = None
     row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
     col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+    fws = torch.empty(max(bsa.forward_workspace_size(B, H, N, d, w.blk), 4), dtype=torch.uint8,
+                      device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
     hp = None
@@ -268,7 +270,7 @@ def run_gpu(args, rank, world, local):
                                   w.stripe_blocks, w.tile_global_frames, row_ptr, col_idx)
 
     def forward():
-        bsa.bsa_forward_into(q, k, v, w.blk, row_ptr, col_idx, o, lse)
+        bsa.bsa_forward_into(q, k, v, w.blk, row_ptr, col_idx, o, lse, workspace=fws)
 
     launches_per_step = (4 if w.source == "asa" else 3) + 1
     for _ in range(args.warmup):

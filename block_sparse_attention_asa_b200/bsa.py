@@ -218,6 +218,10 @@ def pattern_mask_into(head_pattern, B, H, N, blk, band_w, frame_tokens, f_lo, f_
 
 
 # ----------------------------------------------------------------------------- forward
+def forward_workspace_size(B: int, H: int, N: int, d: int, blk: int) -> int:
+    return int(load().bsa_forward_workspace_size(B, H, N, d, blk))
+
+
 def bsa_forward_into(q, k, v, blk, row_ptr, col_idx, o, lse=None, softmax_scale=0.0,
                      workspace=None, stream=None):
     B, H, N, d = _shape(q)
@@ -236,7 +240,7 @@ def bsa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blk: int, row
     B, H, N, d = _shape(q)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    ws_n = int(load().bsa_forward_workspace_size(B, H, N, d, blk))
+    ws_n = forward_workspace_size(B, H, N, d, blk)
     ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
     if col_idx.numel() == 0:
         col_idx = torch.zeros(1, dtype=torch.int32, device=q.device)

@@ -513,22 +513,38 @@ __device__ __forceinline__ void select_row_regs(const float* srow, int i, long l
   if (lane == 0) p.row_ptr[row + 1] = cnt;
 }
 
-// nb <= 32 * NPL <= 1024.  R = rows_per_cta in {8, 16, 32, 64}, nb_pad =
-// 128 * ncb >= kt_ld with (R / 8) * ncb <= 8: warp w owns the 8 x 128 score tile
-// (rows 8 * (w / ncb) .., columns 128 * (w % ncb) ..), a lane 8 rows x 4
-// columns, so one k̄ᵀ float4 and two broadcast q̄ float4 feed 32 FMAs.
-// Shared memory: qs [D][R] fp32, then region A: two stages of dk k̄ᵀ rows
-// (dk * nb_pad floats each), reused for the [R][nb_pad] scores.
-template <int D, int NPL>
-__global__ void __launch_bounds__(256, NPL == 32 ? 2 : 3) asa_select_kernel(const SelectParams p) {
+// Tile shape of asa_select_kernel for nb in (128 (NCB-1), 128 NCB], NCB <= 8.
+template <int D, int NCB>
+struct SelTile {
+  static constexpr int NPL = NCB <= 1 ? 4 : NCB <= 2 ? 8 : NCB <= 4 ? 16 : 32;  // p per lane
+  static constexpr int NB_PAD = 128 * NCB;                 // score row stride
+  static constexpr int R = 8 * (8 / NCB);                  // q-block rows per CTA
+  // k̄ᵀ rows per cp.async stage: a power of two, DK * NB_PAD <= 8192 floats
+  static constexpr int DK = (D * NB_PAD <= 8192) ? D : (D / 2 * NB_PAD <= 8192) ? D / 2
+                            : (D / 4 * NB_PAD <= 8192) ? D / 4 : (D / 8 * NB_PAD <= 8192) ? D / 8
+                            : D / 16;
+  static constexpr int REGION_A = (2 * DK > R ? 2 * DK : R) * NB_PAD;   // floats
+  static constexpr int SMEM = (D * R + REGION_A) * 4;
+  static_assert(DK * NB_PAD <= 8192 && D % DK == 0, "stage size");
+  static_assert((R / 8) * NCB <= 8, "warp tiles");
+};
+
+// nb <= 128 * NCB <= 1024.  R rows per CTA, with (R / 8) * NCB <= 8: warp w
+// owns the 8 x 128 score tile (rows 8 * (w / NCB) .., columns 128 * (w % NCB)
+// ..), a lane 8 rows x 4 columns, so one k̄ᵀ float4 and two broadcast q̄
+// float4 feed 32 FMAs.  Shared memory: qs [D][R] fp32, then region A: two
+// stages of DK k̄ᵀ rows (DK * NB_PAD floats each), reused for the
+// [R][NB_PAD] scores.
+template <int D, int NCB>
+__global__ void __launch_bounds__(256, NCB > 4 ? 2 : 3) asa_select_kernel(const SelectParams p) {
+  using T = SelTile<D, NCB>;
+  constexpr int NPL = T::NPL, R = T::R, nb_pad = T::NB_PAD, DK = T::DK, ncb = NCB;
   extern __shared__ __align__(16) float sel_f[];
-  const int R = p.rows_per_cta, nb_pad = p.nb_pad, DK = p.dk;
   float* qs = sel_f;
   float* ka = sel_f + D * R;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.y, i0 = blockIdx.x * R;
   const int nrow = min(R, p.nb - i0);
-  const int ncb = nb_pad >> 7;
   const int rt = warp / ncb, ct = warp - rt * ncb;
   const bool active = warp < (R >> 3) * ncb && rt * 8 < nrow;
   const float* kt = p.kbarT + (long long)bh * D * p.kt_ld;

@@ -85,7 +85,7 @@ int sm_count() {
 template <int D, int BLK>
 int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
                const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o, float* lse,
-               cudaStream_t stream) {
+               int* item_counter, cudaStream_t stream) {
   using C = FwdCfg<D, BLK>;
   const int nb = (N + BLK - 1) / BLK;
   const int nbw = (nb + 31) / 32;
@@ -118,6 +118,7 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.wait_ns = kWaitNs;
+  p.item_counter = item_counter;
   const int sms = sm_count();
   if (sms <= 0) return BSA_ERR_CUDA;
   // persistent: one CTA per SM, two item slots per CTA
@@ -129,12 +130,12 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
 template <int D>
 int launch_fwd_blk(int blk, const void* q, const void* k, const void* v, int B, int H, int N,
                    const int32_t* rp, const int32_t* ci, float scale, void* o, float* lse,
-                   cudaStream_t s) {
+                   int* ctr, cudaStream_t s) {
   switch (blk) {
-    case 16: return launch_fwd<D, 16>(q, k, v, B, H, N, rp, ci, scale, o, lse, s);
-    case 32: return launch_fwd<D, 32>(q, k, v, B, H, N, rp, ci, scale, o, lse, s);
-    case 64: return launch_fwd<D, 64>(q, k, v, B, H, N, rp, ci, scale, o, lse, s);
-    case 128: return launch_fwd<D, 128>(q, k, v, B, H, N, rp, ci, scale, o, lse, s);
+    case 16: return launch_fwd<D, 16>(q, k, v, B, H, N, rp, ci, scale, o, lse, ctr, s);
+    case 32: return launch_fwd<D, 32>(q, k, v, B, H, N, rp, ci, scale, o, lse, ctr, s);
+    case 64: return launch_fwd<D, 64>(q, k, v, B, H, N, rp, ci, scale, o, lse, ctr, s);
+    case 128: return launch_fwd<D, 128>(q, k, v, B, H, N, rp, ci, scale, o, lse, ctr, s);
   }
   return BSA_ERR_UNSUPPORTED;
 }
@@ -186,22 +187,16 @@ bool allow_smem(K kernel, int bytes, bool (&done)[64]) {
   return true;
 }
 
-template <int D, int NPL>
+template <int D, int NCB>
 int launch_select_regs(bsa::SelectParams sp, int BH, cudaStream_t stream) {
-  // R rows per CTA so that the (R/8) x ncb warp tiles fill at most the 8 warps;
-  // dk = k̄ᵀ rows per stage, a power of two with dk * nb_pad <= 8192 floats.
-  const int ncb = (sp.nb + 127) / 128;
-  sp.nb_pad = ncb * 128;
-  sp.rows_per_cta = 8 * (8 / ncb);
-  int dk = D;
-  while (dk * sp.nb_pad > 8192) dk >>= 1;
-  sp.dk = dk;
-  const size_t region_a = std::max((size_t)2 * dk * sp.nb_pad, (size_t)sp.rows_per_cta * sp.nb_pad);
-  const size_t smem = ((size_t)D * sp.rows_per_cta + region_a) * sizeof(float);
+  using T = bsa::SelTile<D, NCB>;
+  sp.nb_pad = T::NB_PAD;
+  sp.rows_per_cta = T::R;
+  sp.dk = T::DK;
   static bool done[64] = {};
-  if (!allow_smem(bsa::asa_select_kernel<D, NPL>, 112 * 1024, done)) return BSA_ERR_CUDA;
-  dim3 grid(ceil_div(sp.nb, sp.rows_per_cta), BH);
-  bsa::asa_select_kernel<D, NPL><<<grid, 256, smem, stream>>>(sp);
+  if (!allow_smem(bsa::asa_select_kernel<D, NCB>, T::SMEM, done)) return BSA_ERR_CUDA;
+  dim3 grid(ceil_div(sp.nb, T::R), BH);
+  bsa::asa_select_kernel<D, NCB><<<grid, 256, T::SMEM, stream>>>(sp);
   return check_launch() ? BSA_ERR_CUDA : BSA_OK;
 }
 
@@ -244,11 +239,19 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
     sp.mass_tau = tau;
     sp.scale = scale;
     int rc = BSA_OK;
-    if (nb <= 128) rc = launch_select_regs<D, 4>(sp, BH, stream);
-    else if (nb <= 256) rc = launch_select_regs<D, 8>(sp, BH, stream);
-    else if (nb <= 512) rc = launch_select_regs<D, 16>(sp, BH, stream);
-    else if (nb <= 1024) rc = launch_select_regs<D, 32>(sp, BH, stream);
-    else {
+    const int ncb = (nb + 127) / 128;   // 128-column score blocks
+    switch (ncb) {
+      case 1: rc = launch_select_regs<D, 1>(sp, BH, stream); break;
+      case 2: rc = launch_select_regs<D, 2>(sp, BH, stream); break;
+      case 3: rc = launch_select_regs<D, 3>(sp, BH, stream); break;
+      case 4: rc = launch_select_regs<D, 4>(sp, BH, stream); break;
+      case 5: rc = launch_select_regs<D, 5>(sp, BH, stream); break;
+      case 6: rc = launch_select_regs<D, 6>(sp, BH, stream); break;
+      case 7: rc = launch_select_regs<D, 7>(sp, BH, stream); break;
+      case 8: rc = launch_select_regs<D, 8>(sp, BH, stream); break;
+      default: break;
+    }
+    if (ncb > 8) {
       const int nb_pad = (nb + 31) / 32 * 32;
       const size_t budget = 200 * 1024;
       int R = 16;
@@ -404,16 +407,15 @@ int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
 }
 
 size_t bsa_forward_workspace_size(int B, int H, int N, int d, int blk) {
-  (void)B; (void)H; (void)N; (void)d; (void)blk;
-  return 0;
+  if (common_shape_checks(B, H, N, blk) != BSA_OK || (d != 64 && d != 128)) return 0;
+  return 256;   // the item counter of the persistent grid
 }
 
 int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d, int blk,
                 const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale, void* o,
                 float* lse, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
-  (void)workspace;
-  (void)ws_bytes;
   if (!q || !k || !v || !o || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
+  if (workspace != nullptr && (ws_bytes < 4 || !aligned(workspace, 4))) return BSA_ERR_WORKSPACE;
   int rc = common_shape_checks(B, H, N, blk);
   if (rc != BSA_OK) return rc;
   if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
@@ -422,8 +424,12 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
   if (std::isnan(softmax_scale)) return BSA_ERR_INVALID_ARG;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
   cudaStream_t s = as_cuda(stream);
-  if (d == 64) return launch_fwd_blk<64>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, s);
-  return launch_fwd_blk<128>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, s);
+  int* counter = static_cast<int*>(workspace);
+  if (counter != nullptr && cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  if (d == 64)
+    return launch_fwd_blk<64>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);
+  return launch_fwd_blk<128>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);
 }
 
 }  // extern "C"

@@ -15,27 +15,35 @@
 // so that one slot's softmax overlaps the other slot's MMAs.  Items are dealt
 // round-robin: slot X of CTA c takes items 2c+X, 2c+X+2G, ... (G = grid size).
 //
-// Warp roles (384 threads, three warpgroups):
+// Warp roles (640 threads, 20 warps):
 //   warp 3      scheduler: per item builds the q-block bitmaps of its CSR rows
 //               and the ascending union list (block id + keep bits) in shared
-//               memory, double-buffered per slot, and prefetches the item's Q
-//               tile into L2.
+//               memory, in segments, double-buffered per slot, and prefetches
+//               the item's Q tile into L2.
 //   warp 0      producer (one lane, state in registers): per step takes up to
 //               128/blk list entries, publishes a per-slot step entry (ring
 //               index, first/last, block ids, keep bits) and the gathered K
-//               boxes (TMA, 128B swizzle) into a K ring; the V boxes follow on a
-//               separate front, since V is needed one step later than K.
+//               boxes (TMA, 128B swizzle) into a K ring, alternating slots; the
+//               V boxes follow on a separate front, since V is needed one step
+//               later than K.
 //   warps 1, 2  MMA issuers, one thread per slot: S_X = Q_X Kᵀ, then for the
 //               previous step O_X += P_X V with P read from TMEM.  Issuing a
 //               tcgen05.mma costs the issuing thread about as long as the MMA
-//               runs (measured on B200), so each slot has its own issuer.
+//               runs (measured on B200), so each slot has its own issuer; the
+//               two take turns batch by batch so that the slots stay half a
+//               period apart instead of contending for the tensor pipe and
+//               the MUFU at the same time.
 //   warp 2      also allocates and releases TMEM.
-//   warps 4-7   softmax + epilogue of slot A;  warps 8-11 the same for slot B.
-//               Thread = query row = TMEM lane.  Raw-score max (3-input max),
-//               packed f32x2 scale/shift and sums, one ex2 per score, lazy
-//               rescale of O (only when the max grows by more than 2^8; exact
-//               because the final normalisation uses the same stale max),
-//               P (bf16) written over S in TMEM.
+//   warps 4-11  softmax + epilogue of slot A;  warps 12-19 the same for slot B.
+//               Warp (q, h): rows 32q..32q+31 (TMEM lane quarter q), keys
+//               64h..64h+63 of each 128-key step; the two halves of a row
+//               exchange their maxima through shared memory.  Raw-score max
+//               (3-input max), packed f32x2 scale/shift and sums, one ex2 per
+//               score, lazy rescale of O (only when the max grows by more than
+//               2^8; exact because the final normalisation uses the same stale
+//               max), P (bf16) written over S in TMEM.  A half whose keys all
+//               belong to blocks its q-block does not list writes P = 0 without
+//               exponentials.
 //
 // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
 //
@@ -70,6 +78,7 @@ struct FwdParams {
   __nv_bfloat16* o;
   float* lse;
   unsigned long long wait_ns;     // bound on every wait
+  int* item_counter;              // zeroed before launch; null: items dealt statically
 };
 
 template <int D, int BLK>
@@ -90,6 +99,9 @@ struct FwdCfg {
   static constexpr int V_OFF = K_OFF + NK * TILE;
   static constexpr int AUX_OFF = V_OFF + NV * TILE;
   static constexpr int BAR_BYTES = 512;
+  // k/v full+free, q/s/p/o barriers, m_full, l_full+free, drain, pair, issue turn
+  static constexpr int NBARS = 2 * NK + 2 * NV + 12 + 2 * NM + 8 + 2 + 8 + 2;
+  static_assert(NBARS * 8 <= BAR_BYTES, "mbarriers must fit their area");
   static constexpr int SMETA_OFF = AUX_OFF + BAR_BYTES;          // 2 x NM step entries
   static constexpr int SMETA_INTS = 24;
   static constexpr int VQ_INTS = 8 * 12;                         // producer V-front queue
@@ -107,15 +119,20 @@ struct FwdCfg {
 // entry kinds (list headers and per-slot step entries)
 constexpr int kEntryNormal = 0, kEntryEnd = 2;
 
-// 20 warps: 4 control warps, then 8 softmax warps per slot (a row's 128 keys
-// split over two warps that share the row's TMEM lane).
-constexpr int kFwdThreads = 640;
+// Softmax warps per slot: 4 (one per TMEM lane quarter, a thread owns all 128
+// keys of its row) or 8 (two per lane quarter, 64 keys each, the two halves
+// exchanging their row maxima).
+constexpr int kSoftmaxWarps = 8;
+constexpr int kFwdThreads = (4 + 2 * kSoftmaxWarps) * 32;
 // Register split (setmaxnreg, per warpgroup): the control warpgroup (producer,
-// MMA issuers, scheduler) gives registers to the four softmax warpgroups.  The
-// sum must not exceed the launch allocation (640 threads x 96), or the
-// increase would wait forever.
-constexpr int kRegControl = 72, kRegSoftmax = 96;
-static_assert(128 * kRegControl + 512 * kRegSoftmax <= kFwdThreads * 96, "register split over budget");
+// MMA issuers, scheduler) gives registers to the softmax warpgroups.  The sum
+// must not exceed the launch allocation (threads x the per-thread launch
+// limit), or the increase would wait forever.
+constexpr int kLaunchRegs = kSoftmaxWarps == 4 ? 168 : 96;
+constexpr int kRegControl = kSoftmaxWarps == 4 ? 80 : 72;
+constexpr int kRegSoftmax = kSoftmaxWarps == 4 ? 200 : 96;
+static_assert(128 * kRegControl + 2 * kSoftmaxWarps * 32 * kRegSoftmax <= kFwdThreads * kLaunchRegs,
+              "register split over budget");
 
 // list segment header (ints): [0] kind (0 segment, 2 end) [1] bh [2] qt [3] nq
 //                             [4] count [5] first segment [6] last segment
@@ -179,6 +196,9 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // MUFU-bound with idle issue slots; off for now.
 constexpr int kPolyPairs = 0;
 
+// The two slots' MMA issuers alternate batches (see the issuer's comment).
+constexpr bool kAlternateIssue = false;
+
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0, int c1, int c2) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
                    reinterpret_cast<uint64_t>(m)),
@@ -231,10 +251,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* l_free = l_full + 4;                 // [2][2]
   uint64_t* mma_drain = l_free + 4;             // [2]
   uint64_t* pair_bar = mma_drain + 2;            // [2 slots][4 lane quarters]
+  uint64_t* issue_tok = pair_bar + 8;            // [2] MMA issue-order token, per slot
   int* smeta = reinterpret_cast<int*>(smem + C::SMETA_OFF);
   int* hdr = reinterpret_cast<int*>(smem + C::HDR_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   int* abort_flag = reinterpret_cast<int*>(smem + C::MISC_OFF + 4);
+  int* issuer_done = reinterpret_cast<int*>(smem + C::MISC_OFF + 8);   // [2]
   uint32_t* lists = reinterpret_cast<uint32_t*>(smem + C::LIST_OFF);
   uint32_t* bm_all = reinterpret_cast<uint32_t*>(smem + C::BM_OFF);
 
@@ -254,9 +276,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&q_full[x], 1);
       mbar_init(&q_free[x], 1);
       mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], 256);
+      mbar_init(&p_full[x], kSoftmaxWarps);   // one arrive per softmax warp of the slot
       mbar_init(&o_done[x], 1);
-      mbar_init(&o_free[x], 256);
+      mbar_init(&o_free[x], kSoftmaxWarps);
       for (int s = 0; s < C::NM; ++s) mbar_init(&m_full[x * C::NM + s], 1);
       for (int b = 0; b < 2; ++b) {
         mbar_init(&l_full[x * 2 + b], 1);
@@ -265,8 +287,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
     mbar_init(&mma_drain[0], 1);
     mbar_init(&mma_drain[1], 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 64);
+    for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 2);   // one arrive per warp
+    mbar_init(&issue_tok[0], 1);
+    mbar_init(&issue_tok[1], 1);
     *abort_flag = 0;
+    issuer_done[0] = 0;
+    issuer_done[1] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -284,11 +310,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   if (warp == 3) {
     regs_dec<kRegControl>();
     // ================================================================ scheduler
-    // Per slot: next item (round-robin over the grid), its q-block bitmaps,
-    // then the ascending union list in segments of at most LCAP entries.
+    // Per slot: next item, its q-block bitmaps, then the ascending union list
+    // in segments of at most LCAP entries.  Each slot starts on item 2c + X;
+    // later items come from a grid-wide counter, so SMs that run faster take
+    // more items (without a counter: round-robin, 2c + X + 2kG).
     SchedSlot S0, S1;
     S0.item = 2 * blockIdx.x;
     S1.item = 2 * blockIdx.x + 1;
+    auto next_item = [&](int cur) -> int {
+      if (p.item_counter == nullptr) return cur + 2 * static_cast<int>(gridDim.x);
+      int v = 0;
+      if (lane == 0) v = 2 * static_cast<int>(gridDim.x) + atomicAdd(p.item_counter, 1);
+      return __shfl_sync(0xffffffffu, v, 0);
+    };
     uint64_t t_last = global_ns();
     auto publish = [&](SchedSlot& st, int X) -> bool {
       // returns true if a segment (or the end marker) was published
@@ -338,7 +372,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           cnt += __popc(u);
         }
         cnt = warp_sum(cnt);
-        st.item += 2 * (int)gridDim.x;
+        st.item = next_item(st.item);
         if (cnt == 0) {
           // no row of this tile lists anything: O = 0, LSE = -inf
           for (int r = 0; r < 128; ++r) {
@@ -581,12 +615,43 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint32_t t_s = tmem + C::S_COL + X * 128, t_o = tmem + C::O_COL + X * 128;
       int pend = -1, pend_first = 0, pend_last = 0, qc = 0, pc = 0, items = 0;
       bool ok = true, issued = false;
-      auto issue_pv = [&]() -> bool {
+      // The two issuers take turns: a turn is one slot's batch (PV of its
+      // previous step, then QK of its next).  Alternating the batches offsets
+      // the slots by one batch, so one slot's softmax runs while the tensor
+      // pipe serves the other slot, instead of both contending at once.  The
+      // turn order affects speed only; a slot whose partner has finished (or
+      // never started) stops waiting for turns.
+      int tk = 0;
+      bool my_turn = X == 0;
+      auto take_turn = [&]() -> bool {
+        if (!kAlternateIssue) return true;
+        if (my_turn) {
+          my_turn = false;
+          return true;
+        }
+        const uint64_t t0 = global_ns();
+        while (true) {
+          if (mbar_try_wait(&issue_tok[X], tk & 1)) {
+            ++tk;
+            return true;
+          }
+          if (*(volatile int*)&issuer_done[X ^ 1]) return true;
+          if (*(volatile int*)abort_flag) return false;
+          if (global_ns() - t0 > p.wait_ns) return false;
+        }
+      };
+      auto pass_turn = [&]() {
+        if (kAlternateIssue) mbar_arrive(&issue_tok[X ^ 1]);
+      };
+      auto wait_pv = [&]() -> bool {
         const int sp = pend;
         if (!mbar_wait(&v_full[sp % C::NV], (sp / C::NV) & 1, p.wait_ns)) return false;
         if (pend_first && items > 0 && !mbar_wait(&o_free[X], (items - 1) & 1, p.wait_ns))
           return false;
-        if (!mbar_wait(&p_full[X], pc & 1, p.wait_ns)) return false;
+        return mbar_wait(&p_full[X], pc & 1, p.wait_ns);
+      };
+      auto issue_pv = [&]() {
+        const int sp = pend;
         tc_fence_after();
         const uint64_t dv = dv0 + static_cast<uint64_t>(((sp % C::NV) * C::TILE) >> 4);
         const uint32_t acc0 = pend_first ? 0u : 1u;
@@ -601,7 +666,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ++items;
         }
         pend = -1;
-        return true;
       };
       for (int t = 0; ok; ++t) {
         const int mi = X * C::NM + t % C::NM;
@@ -611,11 +675,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int first = sm[1], lastt = sm[2], s = sm[22];
         const int ks = s % C::NK;
         if (!mbar_wait(&k_full[ks], (s / C::NK) & 1, p.wait_ns)) { ok = false; break; }
-        if (pend >= 0 && !issue_pv()) { ok = false; break; }
+        if (pend >= 0 && !wait_pv()) { ok = false; break; }
         if (first) {
           if (!mbar_wait(&q_full[X], qc & 1, p.wait_ns)) { ok = false; break; }
           ++qc;
         }
+        if (!take_turn()) { ok = false; break; }
+        if (pend >= 0) issue_pv();
         tc_fence_after();
         const uint64_t dk = dk0 + static_cast<uint64_t>((ks * C::TILE) >> 4);
 #pragma unroll
@@ -627,11 +693,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mma_commit(&k_free[ks]);
         if (lastt) mma_commit(&q_free[X]);
         mma_commit(&s_full[X]);
+        pass_turn();
         pend = s;
         pend_first = first;
         pend_last = lastt;
       }
-      if (ok && pend >= 0) ok = issue_pv();
+      if (ok && pend >= 0) {
+        ok = wait_pv() && take_turn();
+        if (ok) {
+          issue_pv();
+          pass_turn();
+        }
+      }
+      *(volatile int*)&issuer_done[X] = 1;
       if (!ok) {
         record_error(BSA_ERR_TIMEOUT);
         *(volatile int*)abort_flag = 1;
@@ -645,20 +719,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   } else if (warp >= 4) {
     regs_inc<kRegSoftmax>();
     // ================================================================ softmax
-    // Warps 4-11: slot A, 12-19: slot B.  Warp q + 4h (q = lane quarter,
-    // h = key half) handles rows 32q..32q+31 and keys [64h, 64h+64) of each
-    // step; the two halves of a row agree on the running max through a
-    // shared-memory slot and a two-warp mbarrier (bounded wait).
-    const int X = (warp - 4) >> 3;
-    const int h = ((warp - 4) >> 2) & 1;
+    // kSoftmaxWarps warps per slot (slot A first).  Warp (q, h): q = TMEM lane
+    // quarter (rows 32q..32q+31), h = key part (keys KW*h .. KW*h+KW-1 of each
+    // 128-key step, NH parts).  With two parts, the halves of a row agree on
+    // the running max through shared memory and a two-warp mbarrier.
+    constexpr int NH = kSoftmaxWarps / 4;     // key parts per row
+    constexpr int KW = 128 / NH;              // keys per warp and step
+    constexpr int DW = D / NH;                // O columns per warp in rescale and epilogue
+    const int X = (warp - 4) / kSoftmaxWarps;
+    const int h = ((warp - 4) >> 2) % NH;
     const int wq = warp & 3;                  // TMEM lane quarter
     const int row = wq * 32 + lane;           // query row in the tile
     const int qq = row / BLK;                 // its q-block in the tile
-    uint64_t* pbar = &pair_bar[X * 4 + wq];   // the two warps of this lane quarter
+    uint64_t* pbar = &pair_bar[X * 4 + wq];   // the two warps of this lane quarter (NH = 2)
     int puse = 0;
-    auto pair_sync = [&]() -> bool {
+    // every lane's prior shared-memory writes and tcgen05 operations are
+    // ordered before lane 0's arrive by the warp barrier
+    auto warp_arrive = [&](uint64_t* bar) {
       tc_fence_before();
-      mbar_arrive(pbar);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+    auto pair_sync = [&]() -> bool {
+      warp_arrive(pbar);
       const bool r = mbar_wait(pbar, puse & 1, p.wait_ns);
       ++puse;
       tc_fence_after();
@@ -669,10 +752,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     float* xmax = reinterpret_cast<float*>(smem + C::XCH_OFF);        // [2][2 slots][2 halves][128]
     float* xsum = xmax + 2 * 2 * 2 * 128;                             // [2 slots][2 halves][128]
     const float c2 = p.scale_log2;
-    float m_run = -INFINITY;   // running max of raw scores (same in both halves)
-    float l_run = 0.f;         // this half's running sum
+    float m_run = -INFINITY;   // running max of raw scores (same in every part of a row)
+    float l_run = 0.f;         // this part's running sum
     int items = 0;
     bool ok = true;
+    // kv-block slots overlapping this warp's keys
+    constexpr int SPW = BLK <= KW ? KW / BLK : 1;
+    const int sl0 = BLK <= KW ? h * SPW : 0;
+    const uint32_t warp_mask = ((1u << SPW) - 1u) << sl0;
     for (int t = 0;; ++t) {
       const int mi = X * C::NM + t % C::NM;
       bool w_ok = mbar_wait(&m_full[mi], (t / C::NM) & 1, p.wait_ns) && !*(volatile int*)abort_flag;
@@ -698,12 +785,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
       }
-      // slots overlapping this warp's 64 keys
-      constexpr int SPH = C::SLOTS >= 2 ? C::SLOTS / 2 : 1;    // slots per half
-      const int sl0 = C::SLOTS >= 2 ? h * SPH : 0;
-      const uint32_t half_mask = ((1u << SPH) - 1u) << sl0;
-      const bool live_all = (live_bits & half_mask) == half_mask &&
-                            (part_slot < sl0 || part_slot >= sl0 + SPH);
+      const bool live_all = (live_bits & warp_mask) == warp_mask &&
+                            (part_slot < sl0 || part_slot >= sl0 + SPW);
       if (first) {
         m_run = -INFINITY;
         l_run = 0.f;
@@ -711,40 +794,56 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       w_ok = mbar_wait(&s_full[X], t & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
-      float x[64];
+      // This warp's keys all belong to blocks the row's q-block does not list
+      // (warp-uniform when blk >= 32: a warp's rows share one q-block): no
+      // exponentials, P = 0.
+      const bool part_dead = !__any_sync(0xffffffffu, (live_bits & warp_mask) != 0u);
+      float x[KW];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < KW / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(t_lane + s_col + h * 64 + c * 32, r);
+        tmem_ld32(t_lane + s_col + h * KW + c * 32, r);
 #pragma unroll
         for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
       }
       tmem_wait_ld();
-      // masking: slots this row's q-block does not list, unused slots, keys >= N
-      if (!__all_sync(0xffffffffu, live_all)) {
+      float hmax = -INFINITY;
+      if (!part_dead) {
+        // masking: slots this row's q-block does not list, unused slots, keys >= N
+        if (!__all_sync(0xffffffffu, live_all)) {
+          // valid keys of each block in this warp's range, counted from the
+          // range's first key of that block
+          constexpr int SPAN = BLK < KW ? BLK : KW;
+          int nk_loc[KW / SPAN];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int key = h * 64 + c;             // key index within the step
-          const int sl = key / BLK, e = key % BLK;
-          const int nk = ((live_bits >> sl) & 1u) ? (sl == part_slot ? part_keys : BLK) : 0;
-          if (e >= nk) x[c] = -INFINITY;
+          for (int b = 0; b < KW / SPAN; ++b) {
+            const int sl = BLK <= KW ? sl0 + b : 0;
+            const int nk = ((live_bits >> sl) & 1u) ? (sl == part_slot ? part_keys : BLK) : 0;
+            nk_loc[b] = BLK <= KW ? nk : nk - h * KW;
+          }
+#pragma unroll
+          for (int c = 0; c < KW; ++c)
+            if (c % SPAN >= nk_loc[c / SPAN]) x[c] = -INFINITY;
         }
-      }
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 64; c += 8) {
-        mx0 = fmax3(mx0, x[c], x[c + 1]);
-        mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
-        mx2 = fmax3(mx2, x[c + 4], x[c + 5]);
-        mx3 = fmax3(mx3, x[c + 6], x[c + 7]);
+        for (int c = 0; c < KW; c += 8) {
+          mx0 = fmax3(mx0, x[c], x[c + 1]);
+          mx1 = fmax3(mx1, x[c + 2], x[c + 3]);
+          mx2 = fmax3(mx2, x[c + 4], x[c + 5]);
+          mx3 = fmax3(mx3, x[c + 6], x[c + 7]);
+        }
+        hmax = fmax3(fmax3(mx0, mx1, mx2), mx3, mx3);
       }
-      const float hmax = fmax3(fmax3(mx0, mx1, mx2), mx3, mx3);
-      // agree on the row max with the other half (double-buffered by step
-      // parity); the barrier also orders both halves' S reads before any P write
-      float* xm = xmax + ((t & 1) * 4 + X * 2) * 128;
-      xm[h * 128 + row] = hmax;
-      if (!pair_sync()) { ok = false; break; }
-      const float tmax = fmaxf(hmax, xm[(h ^ 1) * 128 + row]);
+      float tmax = hmax;
+      if (NH > 1) {
+        // agree on the row max with the other half (double-buffered by step
+        // parity); the barrier also orders both halves' S reads before any P write
+        float* xm = xmax + ((t & 1) * 4 + X * 2) * 128;
+        xm[h * 128 + row] = hmax;
+        if (!pair_sync()) { ok = false; break; }
+        tmax = fmaxf(hmax, xm[(h ^ 1) * 128 + row]);
+      }
       // lazy rescale (decided per warp: tcgen05.ld/st are warp-collective)
       const float m_new = fmaxf(m_run, tmax);
       const bool grow = m_run == -INFINITY ? (m_new > -INFINITY) : ((m_new - m_run) * c2 > 8.0f);
@@ -755,15 +854,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (!first && __any_sync(0xffffffffu, grow)) {
         // O_X holds PV up to the previous step, complete (see header); scale
-        // this warp's half of the columns before any PV of this step
+        // this warp's columns before any PV of this step
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < DW / 16; ++c) {
           uint32_t r[16];
-          tmem_ld16(t_lane + o_col + h * (D / 2) + c * 16, r);
+          tmem_ld16(t_lane + o_col + h * DW + c * 16, r);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st16(t_lane + o_col + h * (D / 2) + c * 16, r);
+          tmem_st16(t_lane + o_col + h * DW + c * 16, r);
         }
       }
       const float neg_m = m_run == -INFINITY ? 0.f : -m_run * c2;
@@ -771,54 +870,61 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       uint64_t ls2a = pack2(0.f, 0.f), ls2b = pack2(0.f, 0.f);
       const bool emu = kPolyPairs > 0 && __all_sync(0xffffffffu, live_all);
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
+      for (int q2 = 0; q2 < KW / 32; ++q2) {
         uint32_t pk[16];
+        if (part_dead) {
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int col = q2 * 32 + 2 * c;
-          float a0, a1;
-          unpack2(ffma2(pack2(x[col], x[col + 1]), c2x2, nmx2), a0, a1);
-          float p0, p1;
-          if (emu && (c & 15) >= 16 - kPolyPairs) {
-            p0 = exp2_poly(a0);
-            p1 = exp2_poly(a1);
-          } else {
-            p0 = fast_ex2(a0);
-            p1 = fast_ex2(a1);
+          for (int c = 0; c < 16; ++c) pk[c] = 0u;
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int col = q2 * 32 + 2 * c;
+            float a0, a1;
+            unpack2(ffma2(pack2(x[col], x[col + 1]), c2x2, nmx2), a0, a1);
+            float p0, p1;
+            if (emu && (c & 15) >= 16 - kPolyPairs) {
+              p0 = exp2_poly(a0);
+              p1 = exp2_poly(a1);
+            } else {
+              p0 = fast_ex2(a0);
+              p1 = fast_ex2(a1);
+            }
+            if (c & 1)
+              ls2b = fadd2(ls2b, pack2(p0, p1));
+            else
+              ls2a = fadd2(ls2a, pack2(p0, p1));
+            __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+            pk[c] = *reinterpret_cast<uint32_t*>(&hb);
           }
-          if (c & 1)
-            ls2b = fadd2(ls2b, pack2(p0, p1));
-          else
-            ls2a = fadd2(ls2a, pack2(p0, p1));
-          __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-          pk[c] = *reinterpret_cast<uint32_t*>(&hb);
         }
-        // P (bf16 pairs) over S: keys 64h + 32 q2 .. +31 -> columns 32h + 16 q2
-        tmem_st16(t_lane + s_col + h * 32 + q2 * 16, pk);
+        // P (bf16 pairs) over S: keys KW h + 32 q2 .. +31 -> columns KW/2 h + 16 q2
+        tmem_st16(t_lane + s_col + h * (KW / 2) + q2 * 16, pk);
       }
       float la0, la1, lb0, lb1;
       unpack2(ls2a, la0, la1);
       unpack2(ls2b, lb0, lb1);
       l_run = l_run * alpha + ((la0 + la1) + (lb0 + lb1));
       tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_full[X]);
+      warp_arrive(&p_full[X]);
       if (lastt) {
-        // ---- epilogue of the item: this warp's half of the O columns
+        // ---- epilogue of the item: this warp's O columns
         const int token = e_qt * 128 + row;
         w_ok = mbar_wait(&o_done[X], items & 1, p.wait_ns);
         if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
         tc_fence_after();
-        float* xs = xsum + X * 2 * 128;
-        xs[h * 128 + row] = l_run;
-        if (!pair_sync()) { ok = false; break; }
-        const float l_tot = l_run + xs[(h ^ 1) * 128 + row];
+        float l_tot = l_run;
+        if (NH > 1) {
+          float* xs = xsum + X * 2 * 128;
+          xs[h * 128 + row] = l_run;
+          if (!pair_sync()) { ok = false; break; }
+          l_tot = l_run + xs[(h ^ 1) * 128 + row];
+        }
         const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
-        __nv_bfloat16* orow = p.o + ((long long)e_bh * p.N + token) * D + h * (D / 2);
+        __nv_bfloat16* orow = p.o + ((long long)e_bh * p.N + token) * D + h * DW;
 #pragma unroll 1
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < DW / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(t_lane + o_col + h * (D / 2) + c * 32, r);
+          tmem_ld32(t_lane + o_col + h * DW + c * 32, r);
           tmem_wait_ld();
           uint32_t packed[16];
 #pragma unroll
@@ -835,8 +941,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                   packed[4 * e + 3]);
           }
         }
-        tc_fence_before();
-        mbar_arrive(&o_free[X]);
+        warp_arrive(&o_free[X]);
         if (h == 0 && p.lse != nullptr && token < p.N)
           p.lse[(long long)e_bh * p.N + token] =
               l_tot > 0.f ? (m_run * p.scale + logf(l_tot)) : -INFINITY;
