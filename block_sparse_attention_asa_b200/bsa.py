@@ -16,7 +16,8 @@ from typing import Optional, Sequence, Tuple
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libbsa_b200.so")
+# The in-tree build; BSA_B200_LIB may name another build of the same library.
+LIB_PATH = os.environ.get("BSA_B200_LIB") or os.path.join(_HERE, "libbsa_b200.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "bsa.h")
 
 OK = 0

@@ -9,8 +9,9 @@
 //
 // Kernels, in launch order:
 //   asa_pool_kernel     HBM-bound: streams Q and K once (16-byte loads, fp32
-//                       accumulation in a fixed order), writes q̄ [row][d] and
-//                       k̄ transposed, k̄ᵀ [bh][d][nb padded to 128].
+//                       accumulation in a fixed order, one small CTA per
+//                       block), writes q̄ [row][d] and k̄ transposed,
+//                       k̄ᵀ [bh][d][nb padded to 4].
 //   asa_select_kernel   nb <= 1024.  Per CTA, R q-block rows of one (b, h):
 //                       the score tile S = q̄ k̄ᵀ as a register-blocked fp32
 //                       GEMM (k̄ᵀ streamed through shared memory by cp.async,
@@ -30,34 +31,49 @@
 namespace bsa {
 
 // ------------------------------------------------------------------ pooling
-// One warp per (tensor, b, h, block).  Lane l reads 16 bytes (8 elements) of a
-// row; D/8 lanes cover a row, 256/D rows per warp step.
+// One CTA of kPoolWarps warps per (tensor, b, h, block): warp w sums rows
+// [w*RW, w*RW + RW) of the block (RW = blk / kPoolWarps rounded up), lane l
+// reading 16 bytes (8 elements) of a row, D/8 lanes per row, all of a warp's
+// loads issued before the first add.  Partial sums combine in a fixed order
+// (rows of a lane, then the lanes of a row group by butterfly, then the warps
+// in index order), so the result is deterministic.  Many small CTAs keep the
+// HBM stream even to the last wave.
+constexpr int kPoolWarps = 4;
+
 template <int D>
-__global__ void __launch_bounds__(256) asa_pool_kernel(const __nv_bfloat16* __restrict__ q,
-                                                       const __nv_bfloat16* __restrict__ k,
-                                                       float* __restrict__ qbar,
-                                                       float* __restrict__ kbarT, int BH, int N,
-                                                       int blk, int nb, int kt_ld) {
+__global__ void __launch_bounds__(kPoolWarps * 32) asa_pool_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+    float* __restrict__ qbar, float* __restrict__ kbarT, int BH, int N, int blk, int nb,
+    int kt_ld) {
   constexpr int LPR = D / 8;          // lanes per row
   constexpr int RPS = 32 / LPR;       // rows per warp step
-  const int lane = threadIdx.x & 31;
-  const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  const long long units = 2LL * BH * nb;
-  if (unit >= units) return;
+  __shared__ float part[kPoolWarps][D];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const long long unit = blockIdx.x;
   const bool is_k = unit >= (long long)BH * nb;
   const long long u = is_k ? unit - (long long)BH * nb : unit;
   const long long bh = u / nb;
   const int i = static_cast<int>(u % nb);
   const int r0 = i * blk, nrows = min(blk, N - r0);
+  const int rw = (blk + kPoolWarps - 1) / kPoolWarps;   // rows per warp
+  const int wr0 = warp * rw, wr1 = min(nrows, wr0 + rw);
   const __nv_bfloat16* src = (is_k ? k : q) + (bh * N + r0) * D;
   const int sub = lane / LPR, col = (lane % LPR) * 8;
   float acc[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-#pragma unroll 4
-  for (int r = sub; r < nrows; r += RPS) {
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(src + (long long)r * D + col));
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  // blk <= 128 -> at most 32 rows per warp -> at most 32 / RPS steps
+  constexpr int MAXSTEP = 32 / RPS;
+  uint4 raw[MAXSTEP];
+#pragma unroll
+  for (int s = 0; s < MAXSTEP; ++s) {
+    const int r = wr0 + sub + s * RPS;
+    raw[s] = r < wr1 ? __ldg(reinterpret_cast<const uint4*>(src + (long long)r * D + col))
+                     : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int s = 0; s < MAXSTEP; ++s) {
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[s]);
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const float2 f = __bfloat1622float2(h2[c]);
@@ -71,21 +87,20 @@ __global__ void __launch_bounds__(256) asa_pool_kernel(const __nv_bfloat16* __re
 #pragma unroll
     for (int c = 0; c < 8; ++c) acc[c] += __shfl_xor_sync(0xffffffffu, acc[c], o);
   if (sub == 0) {
-    const float n = static_cast<float>(nrows);
-    if (!is_k) {
-      float4 a, b;
-      a.x = acc[0] / n; a.y = acc[1] / n; a.z = acc[2] / n; a.w = acc[3] / n;
-      b.x = acc[4] / n; b.y = acc[5] / n; b.z = acc[6] / n; b.w = acc[7] / n;
-      float* dst = qbar + u * D + col;
-      reinterpret_cast<float4*>(dst)[0] = a;
-      reinterpret_cast<float4*>(dst)[1] = b;
-    } else {
-      // k̄ᵀ: the CTA's 8 warps pool 8 consecutive blocks, so for each d their
-      // stores fall into one 32-byte sector.
-      float* dst = kbarT + (bh * D + col) * (long long)kt_ld + i;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) dst[(long long)c * kt_ld] = acc[c] / n;
-    }
+    for (int c = 0; c < 8; ++c) part[warp][col + c] = acc[c];
+  }
+  __syncthreads();
+  // warps in index order; thread t < D finishes column t
+  for (int c = threadIdx.x; c < D; c += kPoolWarps * 32) {
+    float v = part[0][c];
+#pragma unroll
+    for (int w = 1; w < kPoolWarps; ++w) v += part[w][c];
+    v /= static_cast<float>(nrows);
+    if (!is_k)
+      qbar[u * D + c] = v;
+    else
+      kbarT[(bh * D + c) * (long long)kt_ld + i] = v;
   }
 }
 

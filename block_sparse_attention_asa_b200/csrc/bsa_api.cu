@@ -215,7 +215,8 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
   // 1. pooling
   {
     const long long units = 2LL * BH * nb;
-    bsa::asa_pool_kernel<D><<<ceil_div(units, 8), 256, 0, stream>>>(
+    if (blk > 32 * bsa::kPoolWarps) return BSA_ERR_UNSUPPORTED;
+    bsa::asa_pool_kernel<D><<<units, bsa::kPoolWarps * 32, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar, kbarT,
         BH, N, blk, nb, static_cast<int>(L.kt_ld));
     if (check_launch()) return BSA_ERR_CUDA;

@@ -29,10 +29,7 @@
 //   warps 1, 2  MMA issuers, one thread per slot: S_X = Q_X Kᵀ, then for the
 //               previous step O_X += P_X V with P read from TMEM.  Issuing a
 //               tcgen05.mma costs the issuing thread about as long as the MMA
-//               runs (measured on B200), so each slot has its own issuer; the
-//               two take turns batch by batch so that the slots stay half a
-//               period apart instead of contending for the tensor pipe and
-//               the MUFU at the same time.
+//               runs (measured on B200), so each slot has its own issuer.
 //   warp 2      also allocates and releases TMEM.
 //   warps 4-11  softmax + epilogue of slot A;  warps 12-19 the same for slot B.
 //               Warp (q, h): rows 32q..32q+31 (TMEM lane quarter q), keys
@@ -53,11 +50,10 @@
 //   * the commit that signals S_X(t) ready also covers PV_X(t-1), issued by
 //     the same thread before QK_X(t), so the softmax may rescale O_X without a
 //     further wait;
-//   * ring index s reuses K and V slots two indices later; the PV that frees
-//     the V slot of an earlier step is issued by its slot's thread as soon as
-//     that thread sees its next step (or its END), which needs only K-front
-//     progress, so the producer never waits on work that needs its own next
-//     step;
+//   * ring index s reuses K and V slots NK and NV indices later; the PV that
+//     frees the V slot of a step is issued by its slot's thread as soon as the
+//     step's P is stored, before that thread waits for anything of its next
+//     step, so the producer never waits on work that needs its own next step;
 //   * a barrier phase is never completed twice before its waiter looks: each
 //     "free" barrier is released only after the front that waits on it has
 //     passed the entry, so every parity wait is unambiguous;
@@ -99,8 +95,8 @@ struct FwdCfg {
   static constexpr int V_OFF = K_OFF + NK * TILE;
   static constexpr int AUX_OFF = V_OFF + NV * TILE;
   static constexpr int BAR_BYTES = 512;
-  // k/v full+free, q/s/p/o barriers, m_full, l_full+free, drain, pair, issue turn
-  static constexpr int NBARS = 2 * NK + 2 * NV + 12 + 2 * NM + 8 + 2 + 8 + 2;
+  // k/v full+free, q/s/p/o barriers, m_full, l_full+free, drain, pair
+  static constexpr int NBARS = 2 * NK + 2 * NV + 12 + 2 * NM + 8 + 2 + 8;
   static_assert(NBARS * 8 <= BAR_BYTES, "mbarriers must fit their area");
   static constexpr int SMETA_OFF = AUX_OFF + BAR_BYTES;          // 2 x NM step entries
   static constexpr int SMETA_INTS = 24;
@@ -196,9 +192,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // MUFU-bound with idle issue slots; off for now.
 constexpr int kPolyPairs = 0;
 
-// The two slots' MMA issuers alternate batches (see the issuer's comment).
-constexpr bool kAlternateIssue = false;
-
 __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0, int c1, int c2) {
   asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
                    reinterpret_cast<uint64_t>(m)),
@@ -251,12 +244,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* l_free = l_full + 4;                 // [2][2]
   uint64_t* mma_drain = l_free + 4;             // [2]
   uint64_t* pair_bar = mma_drain + 2;            // [2 slots][4 lane quarters]
-  uint64_t* issue_tok = pair_bar + 8;            // [2] MMA issue-order token, per slot
   int* smeta = reinterpret_cast<int*>(smem + C::SMETA_OFF);
   int* hdr = reinterpret_cast<int*>(smem + C::HDR_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   int* abort_flag = reinterpret_cast<int*>(smem + C::MISC_OFF + 4);
-  int* issuer_done = reinterpret_cast<int*>(smem + C::MISC_OFF + 8);   // [2]
   uint32_t* lists = reinterpret_cast<uint32_t*>(smem + C::LIST_OFF);
   uint32_t* bm_all = reinterpret_cast<uint32_t*>(smem + C::BM_OFF);
 
@@ -288,11 +279,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(&mma_drain[0], 1);
     mbar_init(&mma_drain[1], 1);
     for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 2);   // one arrive per warp
-    mbar_init(&issue_tok[0], 1);
-    mbar_init(&issue_tok[1], 1);
     *abort_flag = 0;
-    issuer_done[0] = 0;
-    issuer_done[1] = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -615,34 +602,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint32_t t_s = tmem + C::S_COL + X * 128, t_o = tmem + C::O_COL + X * 128;
       int pend = -1, pend_first = 0, pend_last = 0, qc = 0, pc = 0, items = 0;
       bool ok = true, issued = false;
-      // The two issuers take turns: a turn is one slot's batch (PV of its
-      // previous step, then QK of its next).  Alternating the batches offsets
-      // the slots by one batch, so one slot's softmax runs while the tensor
-      // pipe serves the other slot, instead of both contending at once.  The
-      // turn order affects speed only; a slot whose partner has finished (or
-      // never started) stops waiting for turns.
-      int tk = 0;
-      bool my_turn = X == 0;
-      auto take_turn = [&]() -> bool {
-        if (!kAlternateIssue) return true;
-        if (my_turn) {
-          my_turn = false;
-          return true;
-        }
-        const uint64_t t0 = global_ns();
-        while (true) {
-          if (mbar_try_wait(&issue_tok[X], tk & 1)) {
-            ++tk;
-            return true;
-          }
-          if (*(volatile int*)&issuer_done[X ^ 1]) return true;
-          if (*(volatile int*)abort_flag) return false;
-          if (global_ns() - t0 > p.wait_ns) return false;
-        }
-      };
-      auto pass_turn = [&]() {
-        if (kAlternateIssue) mbar_arrive(&issue_tok[X ^ 1]);
-      };
       auto wait_pv = [&]() -> bool {
         const int sp = pend;
         if (!mbar_wait(&v_full[sp % C::NV], (sp / C::NV) & 1, p.wait_ns)) return false;
@@ -668,6 +627,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         pend = -1;
       };
       for (int t = 0; ok; ++t) {
+        // PV of the previous step as soon as its P is stored: it must precede
+        // this step's QK (S_X holds P_X) but need not wait for this step's K
+        if (pend >= 0) {
+          if (!wait_pv()) { ok = false; break; }
+          issue_pv();
+        }
         const int mi = X * C::NM + t % C::NM;
         if (!mbar_wait(&m_full[mi], (t / C::NM) & 1, p.wait_ns)) { ok = false; break; }
         const int* sm = smeta + mi * C::SMETA_INTS;
@@ -675,13 +640,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int first = sm[1], lastt = sm[2], s = sm[22];
         const int ks = s % C::NK;
         if (!mbar_wait(&k_full[ks], (s / C::NK) & 1, p.wait_ns)) { ok = false; break; }
-        if (pend >= 0 && !wait_pv()) { ok = false; break; }
         if (first) {
           if (!mbar_wait(&q_full[X], qc & 1, p.wait_ns)) { ok = false; break; }
           ++qc;
         }
-        if (!take_turn()) { ok = false; break; }
-        if (pend >= 0) issue_pv();
         tc_fence_after();
         const uint64_t dk = dk0 + static_cast<uint64_t>((ks * C::TILE) >> 4);
 #pragma unroll
@@ -693,19 +655,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mma_commit(&k_free[ks]);
         if (lastt) mma_commit(&q_free[X]);
         mma_commit(&s_full[X]);
-        pass_turn();
         pend = s;
         pend_first = first;
         pend_last = lastt;
       }
-      if (ok && pend >= 0) {
-        ok = wait_pv() && take_turn();
-        if (ok) {
-          issue_pv();
-          pass_turn();
-        }
-      }
-      *(volatile int*)&issuer_done[X] = 1;
       if (!ok) {
         record_error(BSA_ERR_TIMEOUT);
         *(volatile int*)abort_flag = 1;

@@ -198,3 +198,19 @@ def test_forward_dense_rows_longer_than_a_list_segment(cuda_lib, blk):
     ci = np.tile(np.arange(nb, dtype=np.int32), nb)
     rows = [0, 1, nb // 2, nb - 2, nb - 1]
     _run_and_compare(cuda_lib, q, k, v, blk, rp, ci, rows=rows)
+
+
+def test_forward_item_order_does_not_change_results(cuda_lib):
+    # with a workspace the CTAs take items from a counter (dynamic order);
+    # without one the items are dealt round-robin: outputs must be identical
+    g = torch.Generator().manual_seed(77)
+    N, d, blk = 9000, 128, 64
+    q, k, v = (torch.randn(1, 4, N, d, generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    nb = -(-N // blk)
+    rp, ci = _random_csr(4 * nb, nb, seed=78, p_empty=0.1, p_full=0.05)
+    rpd, cid = torch.as_tensor(rp).cuda(), torch.as_tensor(ci).cuda()
+    o_dyn, l_dyn = cuda_lib.bsa_forward(q, k, v, blk, rpd, cid)
+    o_st, l_st = torch.empty_like(o_dyn), torch.empty_like(l_dyn)
+    cuda_lib.bsa_forward_into(q, k, v, blk, rpd, cid, o_st, l_st, workspace=None)
+    assert cuda_lib.check_device_status() == 0
+    assert torch.equal(o_dyn, o_st) and torch.equal(l_dyn, l_st)
