@@ -41,6 +41,24 @@ DATASHEET_HBM_GBS = 8000.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes (read + write) per bsa_fwd_kernel launch, from one ncu capture of
+# the bench's own command (profiles/bsa_fwd_kernel_wan.md), keyed by workload and
+# by the sha256 of the kernel source the capture ran: once the kernel changes,
+# the figure no longer applies and the bench reports null.
+FWD_TRAFFIC = {
+    ("wan2.1_1.3b_asa", "d359d527e9cff607c3640e6670e775a8e020761123c91c61e09a6d9754b68da5"):
+        309124608 + 85531392,
+}
+
+
+def fwd_traffic(workload_name: str):
+    import hashlib
+    src = os.path.join(ROOT, "block_sparse_attention_asa_b200", "csrc", "bsa_fwd.cuh")
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    return FWD_TRAFFIC.get((workload_name, sha))
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -362,7 +380,8 @@ def run_gpu(args, rank, world, local):
         "ms_mask": mask_avg, "ms_forward": fwd_avg,
         "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_kind": f"{pk_kind} bf16 burst", "traffic": None,
+                     "peak_kind": f"{pk_kind} bf16 burst", "traffic": fwd_traffic(w.name),
+                     "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "frac_of_sustained": achieved / float(pk.get("bf16_tflops_sustained", peak)),
                      "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS},
         "mask_roofline": {"bound": "hbm", "achieved": mask_gbs, "peak": float(pk["hbm_gbs"]),
