@@ -40,11 +40,11 @@ namespace bsa {
 // HBM stream even to the last wave.
 constexpr int kPoolWarps = 4;
 
-template <int D>
+template <int D, int BLK>
 __global__ void __launch_bounds__(kPoolWarps * 32) asa_pool_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    float* __restrict__ qbar, float* __restrict__ kbarT, int BH, int N, int blk, int nb,
-    int kt_ld) {
+    float* __restrict__ qbar, float* __restrict__ kbarT, int BH, int N, int nb, int kt_ld) {
+  constexpr int blk = BLK;
   constexpr int LPR = D / 8;          // lanes per row
   constexpr int RPS = 32 / LPR;       // rows per warp step
   __shared__ float part[kPoolWarps][D];
@@ -55,15 +55,14 @@ __global__ void __launch_bounds__(kPoolWarps * 32) asa_pool_kernel(
   const long long bh = u / nb;
   const int i = static_cast<int>(u % nb);
   const int r0 = i * blk, nrows = min(blk, N - r0);
-  const int rw = (blk + kPoolWarps - 1) / kPoolWarps;   // rows per warp
+  constexpr int rw = (BLK + kPoolWarps - 1) / kPoolWarps;   // rows per warp
   const int wr0 = warp * rw, wr1 = min(nrows, wr0 + rw);
   const __nv_bfloat16* src = (is_k ? k : q) + (bh * N + r0) * D;
   const int sub = lane / LPR, col = (lane % LPR) * 8;
   float acc[8];
 #pragma unroll
   for (int c = 0; c < 8; ++c) acc[c] = 0.f;
-  // blk <= 128 -> at most 32 rows per warp -> at most 32 / RPS steps
-  constexpr int MAXSTEP = 32 / RPS;
+  constexpr int MAXSTEP = (rw + RPS - 1) / RPS;
   uint4 raw[MAXSTEP];
 #pragma unroll
   for (int s = 0; s < MAXSTEP; ++s) {

@@ -215,10 +215,17 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
   // 1. pooling
   {
     const long long units = 2LL * BH * nb;
-    if (blk > 32 * bsa::kPoolWarps) return BSA_ERR_UNSUPPORTED;
-    bsa::asa_pool_kernel<D><<<units, bsa::kPoolWarps * 32, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), qbar, kbarT,
-        BH, N, blk, nb, static_cast<int>(L.kt_ld));
+    const auto* qq = static_cast<const __nv_bfloat16*>(q);
+    const auto* kk = static_cast<const __nv_bfloat16*>(k);
+    const int ld = static_cast<int>(L.kt_ld);
+    const dim3 g(static_cast<unsigned>(units)), b(bsa::kPoolWarps * 32);
+    switch (blk) {
+      case 16: bsa::asa_pool_kernel<D, 16><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld); break;
+      case 32: bsa::asa_pool_kernel<D, 32><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld); break;
+      case 64: bsa::asa_pool_kernel<D, 64><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld); break;
+      case 128: bsa::asa_pool_kernel<D, 128><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld); break;
+      default: return BSA_ERR_UNSUPPORTED;
+    }
     if (check_launch()) return BSA_ERR_CUDA;
   }
   // 2. scores + selection
