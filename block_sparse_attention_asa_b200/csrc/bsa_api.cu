@@ -119,6 +119,14 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   p.lse = lse;
   p.wait_ns = kWaitNs;
   p.item_counter = item_counter;
+  p.item_order = nullptr;
+  if (item_counter != nullptr) {
+    int* order = reinterpret_cast<int*>(reinterpret_cast<char*>(item_counter) + 256);
+    bsa::fwd_item_order_kernel<<<1, 1024, 0, stream>>>(row_ptr, nb, p.nqt, C::QB, p.n_items, order,
+                                                       item_counter);
+    if (check_launch()) return BSA_ERR_CUDA;
+    p.item_order = order;
+  }
   const int sms = sm_count();
   if (sms <= 0) return BSA_ERR_CUDA;
   // persistent: one CTA per SM, two item slots per CTA
@@ -416,7 +424,9 @@ int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
 
 size_t bsa_forward_workspace_size(int B, int H, int N, int d, int blk) {
   if (common_shape_checks(B, H, N, blk) != BSA_OK || (d != 64 && d != 128)) return 0;
-  return 256;   // the item counter of the persistent grid
+  // the item counter of the persistent grid, then the items' processing order
+  const size_t items = (size_t)B * H * ((N + 127) / 128);
+  return 256 + ((items * sizeof(int) + 255) & ~static_cast<size_t>(255));
 }
 
 int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d, int blk,
@@ -433,8 +443,8 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
   cudaStream_t s = as_cuda(stream);
   int* counter = static_cast<int*>(workspace);
-  if (counter != nullptr && cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess)
-    return BSA_ERR_CUDA;
+  if (counter != nullptr && ws_bytes < bsa_forward_workspace_size(B, H, N, d, blk))
+    return BSA_ERR_WORKSPACE;
   if (d == 64)
     return launch_fwd_blk<64>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);
   return launch_fwd_blk<128>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);

@@ -75,7 +75,60 @@ struct FwdParams {
   float* lse;
   unsigned long long wait_ns;     // bound on every wait
   int* item_counter;              // zeroed before launch; null: items dealt statically
+  const int* item_order;          // processing order of the items; null: index order
 };
+
+// Items in descending order of their listed work (the CSR row lengths of the
+// tile's q-blocks, summed), so that the persistent CTAs take the long items
+// first and the grid's tail holds only short ones; also zeroes the item
+// counter.  One CTA: histogram of the clamped cost, scan, scatter (the order
+// inside a bin follows the atomics, which changes no result).
+constexpr int kOrderBins = 1024;
+__global__ void __launch_bounds__(1024) fwd_item_order_kernel(const int32_t* __restrict__ row_ptr,
+                                                              int nb, int nqt, int qb, int n_items,
+                                                              int* __restrict__ order,
+                                                              int* __restrict__ counter) {
+  __shared__ int hist[kOrderBins];
+  __shared__ int wsum[32];
+  const int t = threadIdx.x;
+  hist[t] = 0;
+  if (t == 0) *counter = 0;
+  __syncthreads();
+  auto bin_of = [&](int it) -> int {
+    const int bh = it / nqt, i0 = (it % nqt) * qb;
+    const long long r0 = (long long)bh * nb + i0;
+    const int i1 = min(i0 + qb, nb);
+    const int cost = row_ptr[r0 + (i1 - i0)] - row_ptr[r0];
+    return kOrderBins - 1 - min(cost, kOrderBins - 1);   // long items first
+  };
+  for (int it = t; it < n_items; it += 1024) atomicAdd(&hist[bin_of(it)], 1);
+  __syncthreads();
+  // exclusive scan of the 1024 bins: warp scans, then the warp totals
+  const int lane = t & 31, w = t >> 5;
+  const int v = hist[t];
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) wsum[w] = incl;
+  __syncthreads();
+  if (w == 0) {
+    const int x = wsum[lane];
+    int xi = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, xi, o);
+      if (lane >= o) xi += u;
+    }
+    wsum[lane] = xi - x;
+  }
+  __syncthreads();
+  hist[t] = wsum[w] + incl - v;   // first slot of bin t
+  __syncthreads();
+  for (int it = t; it < n_items; it += 1024) order[atomicAdd(&hist[bin_of(it)], 1)] = it;
+}
 
 template <int D, int BLK>
 struct FwdCfg {
@@ -248,6 +301,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   int* hdr = reinterpret_cast<int*>(smem + C::HDR_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   int* abort_flag = reinterpret_cast<int*>(smem + C::MISC_OFF + 4);
+  int* mma_lock = reinterpret_cast<int*>(smem + C::MISC_OFF + 8);   // 0 free, X+1 held by slot X
   uint32_t* lists = reinterpret_cast<uint32_t*>(smem + C::LIST_OFF);
   uint32_t* bm_all = reinterpret_cast<uint32_t*>(smem + C::BM_OFF);
 
@@ -280,6 +334,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(&mma_drain[1], 1);
     for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 2);   // one arrive per warp
     *abort_flag = 0;
+    *mma_lock = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -334,8 +389,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ++st.fills;
           return true;
         }
-        st.bh = st.item / p.nqt;
-        st.qt = st.item % p.nqt;
+        const int it = p.item_order != nullptr ? p.item_order[st.item] : st.item;
+        st.bh = it / p.nqt;
+        st.qt = it % p.nqt;
         const int qb0 = st.qt * C::QB;
         st.nq = min(C::QB, p.nb - qb0);
         for (int e = lane; e < C::QB * nbw; e += 32) bm[e] = 0u;
@@ -602,6 +658,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint32_t t_s = tmem + C::S_COL + X * 128, t_o = tmem + C::O_COL + X * 128;
       int pend = -1, pend_first = 0, pend_last = 0, qc = 0, pc = 0, items = 0;
       bool ok = true, issued = false;
+      // A slot's group of MMAs (its PV, or its QK) runs contiguously in the
+      // tensor pipe: the other slot's issuer waits while a group is being
+      // issued.  Interleaved at instruction level, both slots' S would land
+      // late together; grouped, one lands early and the slots drift apart.
+      auto lock_mma = [&]() -> bool {
+        const uint64_t t0 = global_ns();
+        while (atomicCAS(mma_lock, 0, X + 1) != 0) {
+          if (*(volatile int*)abort_flag) return false;
+          if (global_ns() - t0 > p.wait_ns) return false;
+        }
+        return true;
+      };
+      auto unlock_mma = [&]() { atomicExch(mma_lock, 0); };
       auto wait_pv = [&]() -> bool {
         const int sp = pend;
         if (!mbar_wait(&v_full[sp % C::NV], (sp / C::NV) & 1, p.wait_ns)) return false;
@@ -630,8 +699,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // PV of the previous step as soon as its P is stored: it must precede
         // this step's QK (S_X holds P_X) but need not wait for this step's K
         if (pend >= 0) {
-          if (!wait_pv()) { ok = false; break; }
+          if (!wait_pv() || !lock_mma()) { ok = false; break; }
           issue_pv();
+          unlock_mma();
         }
         const int mi = X * C::NM + t % C::NM;
         if (!mbar_wait(&m_full[mi], (t / C::NM) & 1, p.wait_ns)) { ok = false; break; }
@@ -644,6 +714,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (!mbar_wait(&q_full[X], qc & 1, p.wait_ns)) { ok = false; break; }
           ++qc;
         }
+        if (!lock_mma()) { ok = false; break; }
         tc_fence_after();
         const uint64_t dk = dk0 + static_cast<uint64_t>((ks * C::TILE) >> 4);
 #pragma unroll
@@ -655,6 +726,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mma_commit(&k_free[ks]);
         if (lastt) mma_commit(&q_free[X]);
         mma_commit(&s_full[X]);
+        unlock_mma();
         pend = s;
         pend_first = first;
         pend_last = lastt;

@@ -155,11 +155,12 @@ int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
  * Accumulation is fp32 on the tensor cores (tcgen05, operands from TMA-loaded
  * shared memory).  A CSR block id outside [0, nb) is skipped and flagged
  * (BSA_ERR_CSR in the device status).  Workspace: bsa_forward_workspace_size()
- * bytes (256, 4-byte aligned) holding a counter from which the persistent
- * CTAs take work items, so that faster SMs take more; it is zeroed on `stream`
- * before the launch, and concurrent calls need separate workspaces.  NULL is
- * accepted: items are then dealt round-robin.  A non-NULL workspace under 4
- * bytes or misaligned gives BSA_ERR_WORKSPACE. */
+ * bytes, 4-byte aligned: a counter from which the persistent CTAs take work
+ * items (so that faster SMs take more), and the items' processing order, long
+ * items first, computed on `stream` by a small kernel before the main one.
+ * Concurrent calls need separate workspaces.  NULL is accepted: items are
+ * then dealt round-robin in index order.  A non-NULL workspace smaller than
+ * bsa_forward_workspace_size() or misaligned gives BSA_ERR_WORKSPACE. */
 size_t bsa_forward_workspace_size(int B, int H, int N, int d, int blk);
 int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                 int blk, const int32_t* row_ptr, const int32_t* col_idx,

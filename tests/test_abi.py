@@ -36,7 +36,8 @@ def test_workspace_and_capacity_sizes(lib):
     assert bsa.asa_max_nnz(2, 48, 17776, 64, bsa.MODE_TOPK, 33, 0.0, 0, 4) == 2 * 48 * 278 * 37
     assert bsa.asa_max_nnz(1, 2, 128, 16, bsa.MODE_TOPK, 3, 0.0, 1, 0) == 16 * 4
     assert lib.asa_build_mask_workspace_size(1, 1, 100, 96, 16) == 0  # unsupported d
-    assert bsa.forward_workspace_size(1, 12, 32760, 128, 64) == 256     # the item counter
+    # the item counter, then the processing order of the 12 x 256 items
+    assert bsa.forward_workspace_size(1, 12, 32760, 128, 64) == 256 + 12 * 256 * 4
     assert lib.bsa_forward_workspace_size(1, 1, 100, 96, 16) == 0
 
 
@@ -87,6 +88,8 @@ def test_forward_and_pattern_validation(lib):
     bad[13], bad[14] = vp(256), 2
     assert lib.bsa_forward(*bad) == bsa.ERR_WORKSPACE
     bad[13], bad[14] = vp(258), 256
+    assert lib.bsa_forward(*bad) == bsa.ERR_WORKSPACE
+    bad[13], bad[14] = vp(256), 256     # needs 256 + 256 bytes for this shape
     assert lib.bsa_forward(*bad) == bsa.ERR_WORKSPACE
     hp = (ctypes.c_int32 * 2)(0, 9)
     assert lib.pattern_mask(hp, 1, 2, 128, 16, 2, 64, -1, 1, 1, 0, vp(16), vp(16), 8, None,
