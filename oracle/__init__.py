@@ -22,6 +22,10 @@ What it computes, and from where:
 * ``attention`` -- softmax(Q Kᵀ/√d) V per head (Sparse-vDiT blog, "核心公式 /
                    全注意力机制") restricted to the kept blocks, with the
                    log-sum-exp; an empty row (skip head, M1) gives O = 0.
+* ``search``    -- the offline pattern-search quantities of the Sparse-vDiT blog
+                   ("离线搜索损失函数", "注意力模式选择", Algorithm 1): per-head
+                   MSE against full attention, pattern sparsity, the loss
+                   L_i = MSE + lambda (1 - S_i) and the eps selection rule.
 
 Parity pins (``tests/test_oracle_*.py``): dense attention vs torch's float64
 ``scaled_dot_product_attention``; pooling vs ``avg_pool1d``; selection vs
@@ -33,3 +37,4 @@ check against: its parity beyond that is unpinned.
 from .asa import pool, pooled_probs, select_row, asa_mask, MaskInfo  # noqa: F401
 from .patterns import pattern_row, pattern_mask, keep_token_pair  # noqa: F401
 from .attention import masked_attention, attention_rows  # noqa: F401
+from . import search  # noqa: F401
