@@ -46,8 +46,8 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # by the sha256 of the kernel source the capture ran: once the kernel changes,
 # the figure no longer applies and the bench reports null.
 FWD_TRAFFIC = {
-    ("wan2.1_1.3b_asa", "d359d527e9cff607c3640e6670e775a8e020761123c91c61e09a6d9754b68da5"):
-        309124608 + 85531392,
+    ("wan2.1_1.3b_asa", "6bce1d859cba88877f3e4c3efa49d7357392b54369c331678795075c5c8436c3"):
+        310952960 + 85929472,
 }
 
 
@@ -410,7 +410,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="bsa", choices=["bsa", "reference"])
     ap.add_argument("--workload", default="wan", choices=["wan", "cog", "hunyuan", "tiny"])
-    ap.add_argument("--ref-heads", type=int, default=6,
+    ap.add_argument("--ref-heads", type=int, default=12,
                     help="heads in the cpu_baseline sample of the GPU arm")
     ap.add_argument("--ref-heads-per-step", type=int, default=1,
                     help="heads per step of the --impl reference arm")

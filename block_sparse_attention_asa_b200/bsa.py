@@ -52,6 +52,12 @@ _SIGNATURES = {
     "bsa_status_string": (ctypes.c_char_p, [_c_int]),
     "bsa_version": (_c_int, []),
     "bsa_debug_exp2_poly": (_c_int, [_vp, _vp, _c_int, _vp]),
+    "attention_head_mse_workspace_size": (_c_size, [_c_int] * 4),
+    "attention_head_mse": (_c_int, [_vp, _vp] + [_c_int] * 4 + [_vp, _vp, _c_size, _vp]),
+    "csr_head_sparsity_workspace_size": (_c_size, [_c_int]),
+    "csr_head_sparsity": (_c_int, [_vp, _vp] + [_c_int] * 4 + [_vp, _vp, _c_size, _vp]),
+    "pattern_search_select": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, ctypes.c_double,
+                                       ctypes.c_double, _vp, _vp]),
 }
 
 _lib = None
@@ -247,6 +253,49 @@ def bsa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blk: int, row
         col_idx = torch.zeros(1, dtype=torch.int32, device=q.device)
     bsa_forward_into(q, k, v, blk, row_ptr, col_idx, o, lse, softmax_scale, ws, stream)
     return o, lse
+
+
+def head_mse(o_ref: torch.Tensor, o: torch.Tensor, stream=None) -> torch.Tensor:
+    """Per-head MSE(O - O_ref) over all B*N*d elements, float64 [H] on the device."""
+    _need_cuda(o_ref, o)
+    B, H, N, d = _shape(o_ref)
+    lib = load()
+    mse = torch.empty(H, dtype=torch.float64, device=o_ref.device)
+    ws = torch.empty(max(int(lib.attention_head_mse_workspace_size(B, H, N, d)), 256),
+                     dtype=torch.uint8, device=o_ref.device)
+    _check(lib.attention_head_mse(_ptr(o_ref), _ptr(o), B, H, N, d, _ptr(mse), _ptr(ws),
+                                  ws.numel(), _stream(stream)), "attention_head_mse")
+    return mse
+
+
+def head_sparsity(row_ptr: torch.Tensor, col_idx: torch.Tensor, B: int, H: int, N: int, blk: int,
+                  stream=None) -> torch.Tensor:
+    """Per-head fraction of (query, key) token pairs a CSR block mask skips, float64 [H]."""
+    _need_cuda(row_ptr)
+    lib = load()
+    out = torch.empty(H, dtype=torch.float64, device=row_ptr.device)
+    ws = torch.empty(max(int(lib.csr_head_sparsity_workspace_size(H)), 256), dtype=torch.uint8,
+                     device=row_ptr.device)
+    ci = col_idx if col_idx is not None and col_idx.numel() > 0 else None
+    _check(lib.csr_head_sparsity(_ptr(row_ptr), _ptr(ci), B, H, N, blk, _ptr(out), _ptr(ws),
+                                 ws.numel(), _stream(stream)), "csr_head_sparsity")
+    return out
+
+
+def search_select(mse, sparsity, candidates: Sequence[int], lam: float, eps: float):
+    """Sparse-vDiT selection on host arrays mse, sparsity [P, H]:
+    (choice int32 [H], loss float64 [P, H])."""
+    import numpy as np
+    mse = np.ascontiguousarray(mse, dtype=np.float64)
+    sp = np.ascontiguousarray(sparsity, dtype=np.float64)
+    P, H = mse.shape
+    cand = np.ascontiguousarray(candidates, dtype=np.int32)
+    loss = np.empty((P, H), dtype=np.float64)
+    choice = np.empty(H, dtype=np.int32)
+    _check(load().pattern_search_select(mse.ctypes.data, sp.ctypes.data, cand.ctypes.data, P, H,
+                                        float(lam), float(eps), loss.ctypes.data,
+                                        choice.ctypes.data), "pattern_search_select")
+    return choice, loss
 
 
 def debug_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:

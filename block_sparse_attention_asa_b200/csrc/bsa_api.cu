@@ -13,6 +13,7 @@
 #include "pattern.cuh"
 #include "asa_mask.cuh"
 #include "bsa_fwd.cuh"
+#include "search.cuh"
 
 namespace {
 
@@ -119,14 +120,6 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   p.lse = lse;
   p.wait_ns = kWaitNs;
   p.item_counter = item_counter;
-  p.item_order = nullptr;
-  if (item_counter != nullptr) {
-    int* order = reinterpret_cast<int*>(reinterpret_cast<char*>(item_counter) + 256);
-    bsa::fwd_item_order_kernel<<<1, 1024, 0, stream>>>(row_ptr, nb, p.nqt, C::QB, p.n_items, order,
-                                                       item_counter);
-    if (check_launch()) return BSA_ERR_CUDA;
-    p.item_order = order;
-  }
   const int sms = sm_count();
   if (sms <= 0) return BSA_ERR_CUDA;
   // persistent: one CTA per SM, two item slots per CTA
@@ -313,6 +306,83 @@ const char* bsa_status_string(int status) {
   return "unknown status";
 }
 
+// ---- Sparse-vDiT offline search quantities -----------------------------------
+size_t attention_head_mse_workspace_size(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || (d != 64 && d != 128)) return 0;
+  const size_t chunks = (N + bsa::kMseTokens - 1) / bsa::kMseTokens;
+  return (((size_t)B * H * chunks * sizeof(double)) + 255) & ~static_cast<size_t>(255);
+}
+
+int attention_head_mse(const void* o_ref, const void* o, int B, int H, int N, int d, double* mse,
+                       void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  if (!o_ref || !o || !mse) return BSA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || N <= 0) return BSA_ERR_INVALID_ARG;
+  if ((long long)B * H > 65535) return BSA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
+  if (!aligned(o_ref, 16) || !aligned(o, 16) || !aligned(mse, 8)) return BSA_ERR_UNSUPPORTED;
+  const size_t need = attention_head_mse_workspace_size(B, H, N, d);
+  if (!workspace || ws_bytes < need || !aligned(workspace, 256)) return BSA_ERR_WORKSPACE;
+  const int chunks = (N + bsa::kMseTokens - 1) / bsa::kMseTokens;
+  cudaStream_t s = as_cuda(stream);
+  double* partial = static_cast<double*>(workspace);
+  bsa::head_mse_partial_kernel<<<dim3(chunks, B * H), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(o_ref), static_cast<const __nv_bfloat16*>(o), N, d, chunks,
+      partial);
+  if (check_launch()) return BSA_ERR_CUDA;
+  bsa::head_mse_final_kernel<<<ceil_div(H, 128), 128, 0, s>>>(partial, B, H, N, d, chunks, mse);
+  return check_launch();
+}
+
+size_t csr_head_sparsity_workspace_size(int H) {
+  if (H <= 0) return 0;
+  return ((size_t)H * sizeof(unsigned long long) + 255) & ~static_cast<size_t>(255);
+}
+
+int csr_head_sparsity(const int32_t* row_ptr, const int32_t* col_idx, int B, int H, int N, int blk,
+                      double* sparsity, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  if (!row_ptr || !sparsity) return BSA_ERR_INVALID_ARG;
+  int rc = common_shape_checks(B, H, N, blk);
+  if (rc != BSA_OK) return rc;
+  if (!aligned(sparsity, 8)) return BSA_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < csr_head_sparsity_workspace_size(H) || !aligned(workspace, 256))
+    return BSA_ERR_WORKSPACE;
+  const int nb = (N + blk - 1) / blk;
+  const long long rows = (long long)B * H * nb;
+  cudaStream_t s = as_cuda(stream);
+  auto* kept = static_cast<unsigned long long*>(workspace);
+  if (cudaMemsetAsync(kept, 0, (size_t)H * sizeof(unsigned long long), s) != cudaSuccess)
+    return BSA_ERR_CUDA;
+  if (col_idx != nullptr) {
+    bsa::csr_pairs_kernel<<<ceil_div(rows, 8), 256, 0, s>>>(row_ptr, col_idx, H, N, blk, nb, rows,
+                                                            kept);
+    if (check_launch()) return BSA_ERR_CUDA;
+  }
+  bsa::csr_sparsity_final_kernel<<<ceil_div(H, 128), 128, 0, s>>>(kept, B, H, N, sparsity);
+  return check_launch();
+}
+
+int pattern_search_select(const double* mse, const double* sparsity, const int32_t* candidates,
+                          int P, int H, double lambda, double eps, double* loss, int32_t* choice) {
+  if (!mse || !sparsity || !candidates || !choice || P <= 0 || H <= 0) return BSA_ERR_INVALID_ARG;
+  if (std::isnan(lambda) || std::isnan(eps)) return BSA_ERR_INVALID_ARG;
+  for (int h = 0; h < H; ++h) {
+    bool all_above = true;
+    int best = 0;
+    double best_l = 0.0;
+    for (int i = 0; i < P; ++i) {
+      const double l = mse[(size_t)i * H + h] + lambda * (1.0 - sparsity[(size_t)i * H + h]);
+      if (loss) loss[(size_t)i * H + h] = l;
+      if (!(l > eps)) all_above = false;
+      if (i == 0 || l < best_l) {
+        best = i;
+        best_l = l;
+      }
+    }
+    choice[h] = all_above ? BSA_PATTERN_FULL : candidates[best];
+  }
+  return BSA_OK;
+}
+
 int bsa_check_device_status(bsa_stream_t stream) {
   if (cudaStreamSynchronize(as_cuda(stream)) != cudaSuccess) return BSA_ERR_CUDA;
   int v = 0;
@@ -424,9 +494,7 @@ int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
 
 size_t bsa_forward_workspace_size(int B, int H, int N, int d, int blk) {
   if (common_shape_checks(B, H, N, blk) != BSA_OK || (d != 64 && d != 128)) return 0;
-  // the item counter of the persistent grid, then the items' processing order
-  const size_t items = (size_t)B * H * ((N + 127) / 128);
-  return 256 + ((items * sizeof(int) + 255) & ~static_cast<size_t>(255));
+  return 256;   // the item counter of the persistent grid
 }
 
 int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d, int blk,
@@ -443,8 +511,8 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
   cudaStream_t s = as_cuda(stream);
   int* counter = static_cast<int*>(workspace);
-  if (counter != nullptr && ws_bytes < bsa_forward_workspace_size(B, H, N, d, blk))
-    return BSA_ERR_WORKSPACE;
+  if (counter != nullptr && cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess)
+    return BSA_ERR_CUDA;
   if (d == 64)
     return launch_fwd_blk<64>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);
   return launch_fwd_blk<128>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);

@@ -75,60 +75,7 @@ struct FwdParams {
   float* lse;
   unsigned long long wait_ns;     // bound on every wait
   int* item_counter;              // zeroed before launch; null: items dealt statically
-  const int* item_order;          // processing order of the items; null: index order
 };
-
-// Items in descending order of their listed work (the CSR row lengths of the
-// tile's q-blocks, summed), so that the persistent CTAs take the long items
-// first and the grid's tail holds only short ones; also zeroes the item
-// counter.  One CTA: histogram of the clamped cost, scan, scatter (the order
-// inside a bin follows the atomics, which changes no result).
-constexpr int kOrderBins = 1024;
-__global__ void __launch_bounds__(1024) fwd_item_order_kernel(const int32_t* __restrict__ row_ptr,
-                                                              int nb, int nqt, int qb, int n_items,
-                                                              int* __restrict__ order,
-                                                              int* __restrict__ counter) {
-  __shared__ int hist[kOrderBins];
-  __shared__ int wsum[32];
-  const int t = threadIdx.x;
-  hist[t] = 0;
-  if (t == 0) *counter = 0;
-  __syncthreads();
-  auto bin_of = [&](int it) -> int {
-    const int bh = it / nqt, i0 = (it % nqt) * qb;
-    const long long r0 = (long long)bh * nb + i0;
-    const int i1 = min(i0 + qb, nb);
-    const int cost = row_ptr[r0 + (i1 - i0)] - row_ptr[r0];
-    return kOrderBins - 1 - min(cost, kOrderBins - 1);   // long items first
-  };
-  for (int it = t; it < n_items; it += 1024) atomicAdd(&hist[bin_of(it)], 1);
-  __syncthreads();
-  // exclusive scan of the 1024 bins: warp scans, then the warp totals
-  const int lane = t & 31, w = t >> 5;
-  const int v = hist[t];
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int u = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += u;
-  }
-  if (lane == 31) wsum[w] = incl;
-  __syncthreads();
-  if (w == 0) {
-    const int x = wsum[lane];
-    int xi = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int u = __shfl_up_sync(0xffffffffu, xi, o);
-      if (lane >= o) xi += u;
-    }
-    wsum[lane] = xi - x;
-  }
-  __syncthreads();
-  hist[t] = wsum[w] + incl - v;   // first slot of bin t
-  __syncthreads();
-  for (int it = t; it < n_items; it += 1024) order[atomicAdd(&hist[bin_of(it)], 1)] = it;
-}
 
 template <int D, int BLK>
 struct FwdCfg {
@@ -389,9 +336,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           ++st.fills;
           return true;
         }
-        const int it = p.item_order != nullptr ? p.item_order[st.item] : st.item;
-        st.bh = it / p.nqt;
-        st.qt = it % p.nqt;
+        st.bh = st.item / p.nqt;
+        st.qt = st.item % p.nqt;
         const int qb0 = st.qt * C::QB;
         st.nq = min(C::QB, p.nb - qb0);
         for (int e = lane; e < C::QB * nbw; e += 32) bm[e] = 0u;

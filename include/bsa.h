@@ -155,17 +155,49 @@ int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
  * Accumulation is fp32 on the tensor cores (tcgen05, operands from TMA-loaded
  * shared memory).  A CSR block id outside [0, nb) is skipped and flagged
  * (BSA_ERR_CSR in the device status).  Workspace: bsa_forward_workspace_size()
- * bytes, 4-byte aligned: a counter from which the persistent CTAs take work
- * items (so that faster SMs take more), and the items' processing order, long
- * items first, computed on `stream` by a small kernel before the main one.
- * Concurrent calls need separate workspaces.  NULL is accepted: items are
- * then dealt round-robin in index order.  A non-NULL workspace smaller than
- * bsa_forward_workspace_size() or misaligned gives BSA_ERR_WORKSPACE. */
+ * bytes (256, 4-byte aligned) holding a counter from which the persistent
+ * CTAs take work items, so that faster SMs take more; it is zeroed on `stream`
+ * before the launch, and concurrent calls need separate workspaces.  NULL is
+ * accepted: items are then dealt round-robin.  A non-NULL workspace under 4
+ * bytes or misaligned gives BSA_ERR_WORKSPACE. */
 size_t bsa_forward_workspace_size(int B, int H, int N, int d, int blk);
 int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d,
                 int blk, const int32_t* row_ptr, const int32_t* col_idx,
                 float softmax_scale, void* o, float* lse,
                 void* workspace, size_t ws_bytes, bsa_stream_t stream);
+
+/* ---- Sparse-vDiT offline pattern search (diagnostic) ------------------------
+ * Sparse-vDiT blog, "核心公式 / 离线搜索损失函数", "注意力模式选择" and
+ * Algorithm 1: for each head and candidate pattern i,
+ *     L_i = MSE(O_i - O_0) + lambda * (1 - S_i),
+ * O_0 the output of full attention (M0), S_i the pattern's sparsity; the head
+ * keeps full attention when L_i > eps for every candidate, else takes the
+ * candidate of the smallest L_i.  Readings: MSE averages over all B*N*d
+ * elements of the head; S = 1 - (computed query/key token pairs) / (B*N*N),
+ * a kept block pair (i, j) counting n_q(i) * n_k(j) valid tokens; ties go to
+ * the candidate listed first.  The O_i come from bsa_forward on the masks of
+ * pattern_mask; the real search runs on a model's activations, which this
+ * library does not hold.
+ *
+ * attention_head_mse: mse[h] (device, [H] doubles) for bf16 O_ref, O
+ * [B,H,N,d] (device, 16-byte aligned), d in {64, 128}.  Deterministic
+ * (fixed-order sums).  Workspace: attention_head_mse_workspace_size() bytes,
+ * 256-byte aligned.  Asynchronous on `stream`.
+ * csr_head_sparsity: sparsity[h] (device, [H] doubles) of a CSR block mask
+ * over B*H*nb rows (device; each row's block ids ascending, as bsa_forward
+ * requires); col_idx may be NULL when the mask is empty.  Workspace:
+ * csr_head_sparsity_workspace_size(H) bytes, 256-byte aligned.  Asynchronous.
+ * pattern_search_select: host arrays only, no device work.  mse, sparsity
+ * [P][H] (candidate-major), candidates [P] pattern ids; writes choice [H]
+ * (a candidate id or BSA_PATTERN_FULL) and, when loss is not NULL, L [P][H]. */
+size_t attention_head_mse_workspace_size(int B, int H, int N, int d);
+int attention_head_mse(const void* o_ref, const void* o, int B, int H, int N, int d, double* mse,
+                       void* workspace, size_t ws_bytes, bsa_stream_t stream);
+size_t csr_head_sparsity_workspace_size(int H);
+int csr_head_sparsity(const int32_t* row_ptr, const int32_t* col_idx, int B, int H, int N, int blk,
+                      double* sparsity, void* workspace, size_t ws_bytes, bsa_stream_t stream);
+int pattern_search_select(const double* mse, const double* sparsity, const int32_t* candidates,
+                          int P, int H, double lambda, double eps, double* loss, int32_t* choice);
 
 /* ---- status ----------------------------------------------------------------
  * bsa_check_device_status synchronizes `stream`, returns the first error any

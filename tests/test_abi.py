@@ -36,8 +36,7 @@ def test_workspace_and_capacity_sizes(lib):
     assert bsa.asa_max_nnz(2, 48, 17776, 64, bsa.MODE_TOPK, 33, 0.0, 0, 4) == 2 * 48 * 278 * 37
     assert bsa.asa_max_nnz(1, 2, 128, 16, bsa.MODE_TOPK, 3, 0.0, 1, 0) == 16 * 4
     assert lib.asa_build_mask_workspace_size(1, 1, 100, 96, 16) == 0  # unsupported d
-    # the item counter, then the processing order of the 12 x 256 items
-    assert bsa.forward_workspace_size(1, 12, 32760, 128, 64) == 256 + 12 * 256 * 4
+    assert bsa.forward_workspace_size(1, 12, 32760, 128, 64) == 256     # the item counter
     assert lib.bsa_forward_workspace_size(1, 1, 100, 96, 16) == 0
 
 
@@ -89,8 +88,6 @@ def test_forward_and_pattern_validation(lib):
     assert lib.bsa_forward(*bad) == bsa.ERR_WORKSPACE
     bad[13], bad[14] = vp(258), 256
     assert lib.bsa_forward(*bad) == bsa.ERR_WORKSPACE
-    bad[13], bad[14] = vp(256), 256     # needs 256 + 256 bytes for this shape
-    assert lib.bsa_forward(*bad) == bsa.ERR_WORKSPACE
     hp = (ctypes.c_int32 * 2)(0, 9)
     assert lib.pattern_mask(hp, 1, 2, 128, 16, 2, 64, -1, 1, 1, 0, vp(16), vp(16), 8, None,
                             None) == bsa.ERR_INVALID_ARG
@@ -101,3 +98,38 @@ def test_forward_and_pattern_validation(lib):
                             None) == bsa.ERR_INVALID_ARG
     assert lib.pattern_mask(None, 1, 2, 128, 16, 2, 64, -1, 1, 1, 0, vp(16), vp(16), 8, None,
                             None) == bsa.ERR_INVALID_ARG
+
+
+def test_search_entry_points_validate_and_select_on_host(lib):
+    import numpy as np
+    from oracle import search
+    vp = ctypes.c_void_p
+    dv = ctypes.c_double
+    # host validation (nothing launched)
+    assert lib.attention_head_mse(None, vp(256), 1, 1, 64, 64, vp(256), vp(256), 1024,
+                                  None) == bsa.ERR_INVALID_ARG
+    assert lib.attention_head_mse(vp(256), vp(256), 1, 1, 64, 96, vp(256), vp(256), 1024,
+                                  None) == bsa.ERR_UNSUPPORTED
+    assert lib.attention_head_mse(vp(256), vp(256), 1, 1, 64, 64, vp(256), vp(256), 8,
+                                  None) == bsa.ERR_WORKSPACE
+    assert lib.csr_head_sparsity(vp(256), vp(256), 1, 2, 64, 24, vp(256), vp(256), 256,
+                                 None) == bsa.ERR_UNSUPPORTED
+    assert lib.csr_head_sparsity(vp(256), vp(256), 1, 2, 64, 16, vp(256), None, 0,
+                                 None) == bsa.ERR_WORKSPACE
+    assert lib.attention_head_mse_workspace_size(1, 12, 32760, 128) == 12 * 512 * 8
+    # the selection itself is host code: parity with the oracle's rule
+    rng = np.random.default_rng(3)
+    for trial in range(20):
+        P, H = 4, 9
+        mse = rng.uniform(0, 0.2, (P, H))
+        sp = rng.uniform(0, 1, (P, H))
+        sp[0] = 1.0
+        if trial % 5 == 0:
+            mse[1] = mse[2]           # exact ties
+            sp[1] = sp[2]
+        cand = [1, 2, 3, 4]
+        lam, eps = 0.01 * (trial % 3 + 1), 0.02 * (trial % 4 + 1)
+        choice, loss = bsa.search_select(mse, sp, cand, lam, eps)
+        ref_l = search.search_loss(mse, sp, lam)
+        np.testing.assert_allclose(loss, ref_l, rtol=0, atol=0)
+        assert choice.tolist() == search.select_pattern(ref_l, cand, eps).tolist()
