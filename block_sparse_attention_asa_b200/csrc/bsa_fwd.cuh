@@ -54,6 +54,10 @@
 //     frees the V slot of a step is issued by its slot's thread as soon as the
 //     step's P is stored, before that thread waits for anything of its next
 //     step, so the producer never waits on work that needs its own next step;
+//   * the producer blocks only on the scheduler (list segments); what needs
+//     consumer progress -- a free K slot, the slot's Q buffer after its item's
+//     last QK -- is polled, because that progress may itself wait for a V tile
+//     that only this thread's V front loads;
 //   * a barrier phase is never completed twice before its waiter looks: each
 //     "free" barrier is released only after the front that waits on it has
 //     passed the entry, so every parity wait is unambiguous;
@@ -100,7 +104,8 @@ struct FwdCfg {
   static_assert(NBARS * 8 <= BAR_BYTES, "mbarriers must fit their area");
   static constexpr int SMETA_OFF = AUX_OFF + BAR_BYTES;          // 2 x NM step entries
   static constexpr int SMETA_INTS = 24;
-  static constexpr int VQ_INTS = 8 * 12;                         // producer V-front queue
+  static constexpr int VQ = 8;                                   // V-front queue entries
+  static constexpr int VQ_INTS = VQ * 12;                        // producer V-front queue
   static constexpr int HDR_OFF = SMETA_OFF + (2 * NM * SMETA_INTS + VQ_INTS) * 4;  // 2x2 headers x 8 ints
   static constexpr int MISC_OFF = HDR_OFF + 2 * 2 * 8 * 4;
   static constexpr int LIST_OFF = MISC_OFF + 64;                 // 2 slots x 2 bufs x LCAP
@@ -207,6 +212,7 @@ struct ProdSlot {
   int tcount = 0;     // softmax entries published
   int qcount = 0;     // Q tiles loaded
   bool have = false, lastseg = false, first_tile = false, flushed = false;
+  bool need_q = false;  // the current item's Q tile is not loaded yet
 };
 
 // Scheduler state of one item slot.
@@ -452,9 +458,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int* vq = smeta + 2 * C::NM * C::SMETA_INTS;   // V-front queue: 8 entries x 12 ints
       // One K-front entry for slot X.  Returns false on a wait that gave up.
       bool used_ring = false;
+      bool k_stalled = false;
       auto k_step = [&](ProdSlot& P, int X) -> bool {
         used_ring = false;
-        int* vqe = vq + (sk & 7) * 12;
+        k_stalled = false;
+        int* vqe = vq + (sk % C::VQ) * 12;
         if (!P.have || P.pos == P.count) {
           if (P.have) {
             mbar_arrive(&l_free[X * 2 + ((P.sc - 1) & 1)]);
@@ -482,15 +490,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             P.qt = h[2];
             P.nq = h[3];
             P.first_tile = true;
-            // Q tile (after the previous item's last QK on this slot)
-            if (P.qcount > 0 && !mbar_wait(&q_free[X], (P.qcount - 1) & 1, p.wait_ns)) return false;
-            mbar_arrive_expect_tx(&q_full[X], C::TILE);
-#pragma unroll
-            for (int c = 0; c < C::NCH; ++c)
-              tma_load_3d(smem + C::Q_OFF + X * C::TILE + c * C::CHUNK, &tm_q, &q_full[X], c * 64,
-                          P.qt * 128, P.bh);
-            ++P.qcount;
+            P.need_q = true;
           }
+        }
+        if (P.need_q) {
+          // Q tile, after the previous item's last QK on this slot.  Polled, not
+          // waited for: that QK follows a PV whose V tile this same thread's V
+          // front may still have to load.
+          if (P.qcount > 0 && !mbar_try_wait(&q_free[X], (P.qcount - 1) & 1)) {
+            k_stalled = true;
+            return true;
+          }
+          mbar_arrive_expect_tx(&q_full[X], C::TILE);
+#pragma unroll
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(smem + C::Q_OFF + X * C::TILE + c * C::CHUNK, &tm_q, &q_full[X], c * 64,
+                        P.qt * 128, P.bh);
+          ++P.qcount;
+          P.need_q = false;
         }
         const uint32_t* list = lists + (X * 2 + ((P.sc - 1) & 1)) * C::LCAP;
         int* sm = smeta + (X * C::NM + P.tcount % C::NM) * C::SMETA_INTS;
@@ -535,7 +552,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (*(volatile int*)abort_flag) break;
         bool prog = false;
         // ---- K front
-        if (!k_done && (sk < C::NK || mbar_try_wait(&k_free[sk % C::NK], ((sk / C::NK) - 1) & 1))) {
+        // (the K front stays less than VQ entries ahead of the V front, whose
+        // queue entry it writes)
+        if (!k_done && sk - sv < C::VQ &&
+            (sk < C::NK || mbar_try_wait(&k_free[sk % C::NK], ((sk / C::NK) - 1) & 1))) {
           int X = last ^ 1;
           const bool f0 = P0.flushed, f1 = P1.flushed;
           if ((X == 0 && f0) || (X == 1 && f1)) X ^= 1;
@@ -544,14 +564,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           } else {
             ok = (X == 0) ? k_step(P0, 0) : k_step(P1, 1);
             if (!ok) break;
-            last = X;
-            if (used_ring) ++sk;
+            if (!k_stalled) {   // a stalled slot is retried next, keeping the order
+              last = X;
+              if (used_ring) ++sk;
+              prog = true;
+            }
           }
-          prog = true;
+          if (k_done) prog = true;
         }
         // ---- V front
         while (sv < sk && (sv < C::NV || mbar_try_wait(&v_free[sv % C::NV], ((sv / C::NV) - 1) & 1))) {
-          const int* vqe = vq + (sv & 7) * 12;
+          const int* vqe = vq + (sv % C::VQ) * 12;
           const int vs = sv % C::NV;
           mbar_arrive_expect_tx(&v_full[vs], C::TILE);
 #pragma unroll

@@ -214,3 +214,33 @@ def test_forward_item_order_does_not_change_results(cuda_lib):
     cuda_lib.bsa_forward_into(q, k, v, blk, rpd, cid, o_st, l_st, workspace=None)
     assert cuda_lib.check_device_status() == 0
     assert torch.equal(o_dyn, o_st) and torch.equal(l_dyn, l_st)
+
+
+def test_forward_back_to_back_layers_finish_cleanly(cuda_lib):
+    # The CogVideoX-shaped layer (d 64: 4-deep K/V rings) run as the bench runs
+    # it, mask then forward, many times: every launch must finish with no
+    # device-side wait giving up (a producer that blocked on a Q buffer while
+    # its own V front owed the data that frees it once timed out here).
+    w = W.COG
+    q, k, v = (t.cuda() for t in W.make_qkv(w))
+    B, H, N, d = q.shape
+    cap = cuda_lib.asa_max_nnz(B, H, N, w.blk, w.mode, w.topk, w.max_keep_ratio, w.keep_diag,
+                               w.n_sink_blocks)
+    rp = torch.empty(B * H * w.nb + 1, dtype=torch.int32, device="cuda")
+    ci = torch.empty(cap, dtype=torch.int32, device="cuda")
+    ws = torch.empty(cuda_lib.asa_workspace_size(B, H, N, d, w.blk), dtype=torch.uint8,
+                     device="cuda")
+    fws = torch.empty(cuda_lib.forward_workspace_size(B, H, N, d, w.blk), dtype=torch.uint8,
+                      device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device="cuda")
+    ref = None
+    for it in range(60):
+        cuda_lib.asa_build_mask_into(q, k, w.blk, w.mode, w.topk, w.mass_tau, w.max_keep_ratio,
+                                     w.keep_diag, w.n_sink_blocks, 0.0, rp, ci, ws)
+        cuda_lib.bsa_forward_into(q, k, v, w.blk, rp, ci, o, lse, workspace=fws)
+        assert cuda_lib.check_device_status() == 0, f"iteration {it}"
+        if ref is None:
+            ref = o.clone()
+        elif it % 10 == 0:
+            assert torch.equal(o, ref)
