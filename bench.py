@@ -46,8 +46,8 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 # by the sha256 of the kernel source the capture ran: once the kernel changes,
 # the figure no longer applies and the bench reports null.
 FWD_TRAFFIC = {
-    ("wan2.1_1.3b_asa", "6bce1d859cba88877f3e4c3efa49d7357392b54369c331678795075c5c8436c3"):
-        310952960 + 85929472,
+    ("wan2.1_1.3b_asa", "96289554c31f2322f6a5e5b32e686dc6dd3aafabd8be7fdf376cfb7edc0f9c88"):
+        309146368 + 85984768,
 }
 
 

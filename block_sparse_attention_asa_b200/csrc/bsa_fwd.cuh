@@ -54,10 +54,10 @@
 //     frees the V slot of a step is issued by its slot's thread as soon as the
 //     step's P is stored, before that thread waits for anything of its next
 //     step, so the producer never waits on work that needs its own next step;
-//   * the producer blocks only on the scheduler (list segments); what needs
-//     consumer progress -- a free K slot, the slot's Q buffer after its item's
-//     last QK -- is polled, because that progress may itself wait for a V tile
-//     that only this thread's V front loads;
+//   * the producer never stops its V front while it waits on consumer
+//     progress (a free K slot is polled; the slot's Q buffer, released by its
+//     item's last QK, is waited for with the V front running), because that
+//     progress may itself need a V tile only this thread's V front loads;
 //   * a barrier phase is never completed twice before its waiter looks: each
 //     "free" barrier is released only after the front that waits on it has
 //     passed the entry, so every parity wait is unambiguous;
@@ -458,10 +458,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int* vq = smeta + 2 * C::NM * C::SMETA_INTS;   // V-front queue: 8 entries x 12 ints
       // One K-front entry for slot X.  Returns false on a wait that gave up.
       bool used_ring = false;
-      bool k_stalled = false;
+      // One pass of the V front: loads every V tile whose slot is free.
+      auto v_front = [&]() -> bool {
+        bool moved = false;
+        while (sv < sk && (sv < C::NV || mbar_try_wait(&v_free[sv % C::NV], ((sv / C::NV) - 1) & 1))) {
+          const int* vqe = vq + (sv % C::VQ) * 12;
+          const int vs = sv % C::NV;
+          mbar_arrive_expect_tx(&v_full[vs], C::TILE);
+#pragma unroll
+          for (int sl = 0; sl < C::SLOTS; ++sl)
+#pragma unroll
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_3d(smem + C::V_OFF + vs * C::TILE + c * C::CHUNK + sl * BLK * 128, &tm_v,
+                          &v_full[vs], c * 64, vqe[2 + sl] * BLK, vqe[1]);
+          ++sv;
+          moved = true;
+        }
+        return moved;
+      };
       auto k_step = [&](ProdSlot& P, int X) -> bool {
         used_ring = false;
-        k_stalled = false;
         int* vqe = vq + (sk % C::VQ) * 12;
         if (!P.have || P.pos == P.count) {
           if (P.have) {
@@ -494,12 +510,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
         if (P.need_q) {
-          // Q tile, after the previous item's last QK on this slot.  Polled, not
-          // waited for: that QK follows a PV whose V tile this same thread's V
-          // front may still have to load.
+          // Q tile, after the previous item's last QK on this slot.  While
+          // waiting, keep the V front going: that QK follows a PV whose V tile
+          // this same thread's V front may still have to load.
           if (P.qcount > 0 && !mbar_try_wait(&q_free[X], (P.qcount - 1) & 1)) {
-            k_stalled = true;
-            return true;
+            const uint64_t t0 = global_ns();
+            while (!mbar_try_wait(&q_free[X], (P.qcount - 1) & 1)) {
+              v_front();
+              if (global_ns() - t0 > p.wait_ns) return false;
+            }
           }
           mbar_arrive_expect_tx(&q_full[X], C::TILE);
 #pragma unroll
@@ -564,28 +583,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           } else {
             ok = (X == 0) ? k_step(P0, 0) : k_step(P1, 1);
             if (!ok) break;
-            if (!k_stalled) {   // a stalled slot is retried next, keeping the order
-              last = X;
-              if (used_ring) ++sk;
-              prog = true;
-            }
+            last = X;
+            if (used_ring) ++sk;
           }
-          if (k_done) prog = true;
-        }
-        // ---- V front
-        while (sv < sk && (sv < C::NV || mbar_try_wait(&v_free[sv % C::NV], ((sv / C::NV) - 1) & 1))) {
-          const int* vqe = vq + (sv % C::VQ) * 12;
-          const int vs = sv % C::NV;
-          mbar_arrive_expect_tx(&v_full[vs], C::TILE);
-#pragma unroll
-          for (int sl = 0; sl < C::SLOTS; ++sl)
-#pragma unroll
-            for (int c = 0; c < C::NCH; ++c)
-              tma_load_3d(smem + C::V_OFF + vs * C::TILE + c * C::CHUNK + sl * BLK * 128, &tm_v,
-                          &v_full[vs], c * 64, vqe[2 + sl] * BLK, vqe[1]);
-          ++sv;
           prog = true;
         }
+        // ---- V front
+        if (v_front()) prog = true;
         if (k_done && sv == sk) break;
         if (prog) {
           t_last = global_ns();
