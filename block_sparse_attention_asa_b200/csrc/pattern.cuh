@@ -10,7 +10,8 @@
 // One warp per (h, q-block): lanes sweep the candidate kv-blocks, a ballot and
 // a popcount prefix give each kept block its position, and the row is written
 // once per batch index (the pattern does not depend on b).  Count pass, scan,
-// write pass.  The output is write-bound.
+// write pass.  Full and diagonal rows are contiguous ranges and skip the
+// per-block test; the output is write-bound.
 #pragma once
 #include "common.cuh"
 
@@ -27,11 +28,6 @@ struct PatternParams {
   int8_t head_pattern[kMaxPatternHeads];
 };
 
-__device__ __forceinline__ long long floor_div(long long a, long long b) {
-  long long q = a / b;
-  return (a % b != 0 && ((a < 0) != (b < 0))) ? q - 1 : q;
-}
-
 // Is kv-block j kept for q-block i under `pattern`?
 __device__ __forceinline__ bool pattern_keep(const PatternParams& p, int pattern, int i, int j) {
   switch (pattern) {
@@ -44,25 +40,37 @@ __device__ __forceinline__ bool pattern_keep(const PatternParams& p, int pattern
     default:
       break;
   }
-  const long long blk = p.blk, S = p.frame_tokens;
-  const long long ti_lo = (long long)i * blk, ti_hi = min((long long)p.N, ti_lo + blk) - 1;
-  const long long uj_lo = (long long)j * blk, uj_hi = min((long long)p.N, uj_lo + blk) - 1;
+  // token ranges of the two blocks (N < 2^31, so 32-bit arithmetic is exact)
+  const int blk = p.blk, S = p.frame_tokens;
+  const int ti_lo = i * blk, ti_hi = min(p.N, ti_lo + blk) - 1;
+  const int uj_lo = j * blk, uj_hi = min(p.N, uj_lo + blk) - 1;
   if (pattern == BSA_PATTERN_MULTIDIAG) {
-    // offsets u - t over the two blocks: [lo, hi]; a frame offset f is hit when
-    // [lo, hi] meets [f*S - w*blk, f*S + w*blk]
-    const long long lo = uj_lo - ti_hi, hi = uj_hi - ti_lo, wb = (long long)p.band_w * blk;
-    long long fmin = -floor_div(-(lo - wb), S);  // ceil((lo - wb) / S)
-    long long fmax = floor_div(hi + wb, S);
+    // offsets u - t over the two blocks: [lo, hi]; frame offset f is hit when
+    // [lo, hi] meets [f*S - w*blk, f*S + w*blk] (a few f: no division)
+    const long long lo = (long long)uj_lo - ti_hi, hi = (long long)uj_hi - ti_lo;
+    const long long wb = (long long)p.band_w * blk;
+    if (p.f_hi - p.f_lo <= 8) {
+      for (int f = p.f_lo; f <= p.f_hi; ++f) {
+        const long long c = (long long)f * S;
+        if (lo <= c + wb && hi >= c - wb) return true;
+      }
+      return false;
+    }
+    // many offsets: the f range that [lo, hi] can reach, in closed form
+    const long long a = lo - wb, bb = hi + wb;
+    long long fmin = a >= 0 ? (a + S - 1) / S : -((-a) / S);    // ceil(a / S)
+    long long fmax = bb >= 0 ? bb / S : -((-bb + S - 1) / S);   // floor(bb / S)
     fmin = max(fmin, (long long)p.f_lo);
     fmax = min(fmax, (long long)p.f_hi);
     return fmin <= fmax;
   }
   if (pattern == BSA_PATTERN_STRIPE) {
-    const long long f = uj_lo / S;
-    return (uj_lo - f * S) < (long long)p.stripe_blocks * blk || (f + 1) * S <= uj_hi;
+    const int f = uj_lo / S;
+    return (long long)(uj_lo - f * S) < (long long)p.stripe_blocks * blk ||
+           (long long)(f + 1) * S <= uj_hi;
   }
   if (pattern == BSA_PATTERN_TILE3D) {
-    const long long fi_lo = ti_lo / S, fi_hi = ti_hi / S, fj_lo = uj_lo / S, fj_hi = uj_hi / S;
+    const int fi_lo = ti_lo / S, fi_hi = ti_hi / S, fj_lo = uj_lo / S, fj_hi = uj_hi / S;
     return (fj_lo <= fi_hi && fj_hi >= fi_lo) || fj_lo < p.tile_global_frames;
   }
   return false;
@@ -103,26 +111,29 @@ __global__ void __launch_bounds__(256) pattern_kernel(const __grid_constant__ Pa
       for (int b = 0; b < p.B; ++b) p.row_ptr[((long long)b * p.H + h) * p.nb + i + 1] = cnt;
     return;
   }
-  const int nbatch = p.B;
-  int pos = 0;
-  for (int jb = j0; jb < j1; jb += 32) {
-    const int j = jb + lane;
-    const bool keep = j < j1 && pattern_keep(p, pattern, i, j);
-    const unsigned m = __ballot_sync(0xffffffffu, keep);
-    const int off = pos + __popc(m & ((1u << lane) - 1u));
-    if (keep) {
-      for (int b = 0; b < nbatch; ++b) {
-        const long long r = ((long long)b * p.H + h) * p.nb + i;
-        const long long at = (long long)p.row_ptr[r] + off;
-        if (at < p.row_ptr[r + 1]) {
+  // Full and diagonal rows are one contiguous range: no per-block test.  The
+  // row's bounds are read once per batch index, outside the block sweep.
+  const bool contiguous = pattern == BSA_PATTERN_FULL || pattern == BSA_PATTERN_DIAG;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int b = 0; b < p.B; ++b) {
+    const long long r = ((long long)b * p.H + h) * p.nb + i;
+    const long long base = p.row_ptr[r], end = p.row_ptr[r + 1];
+    int pos = 0;
+    for (int jb = j0; jb < j1; jb += 32) {
+      const int j = jb + lane;
+      const bool keep = j < j1 && (contiguous || pattern_keep(p, pattern, i, j));
+      const unsigned m = __ballot_sync(0xffffffffu, keep);
+      if (keep) {
+        const long long at = base + pos + __popc(m & lt);
+        if (at < end) {
           if (at < p.capacity)
             p.col_idx[at] = j;
           else
             record_error(BSA_ERR_CAPACITY);
         }
       }
+      pos += __popc(m);
     }
-    pos += __popc(m);
   }
 }
 
