@@ -22,6 +22,10 @@ What it computes, and from where:
 * ``attention`` -- softmax(Q Kᵀ/√d) V per head (Sparse-vDiT blog, "核心公式 /
                    全注意力机制") restricted to the kept blocks, with the
                    log-sum-exp; an empty row (skip head, M1) gives O = 0.
+* ``backward``  -- dQ, dK, dV of the masked attention for a given dO (BLADE
+                   digest, "技术框架": ASA is trained jointly, so the attention is
+                   differentiated; the mask is a constant of the step), and the
+                   transpose of a CSR block mask.
 * ``search``    -- the offline pattern-search quantities of the Sparse-vDiT blog
                    ("离线搜索损失函数", "注意力模式选择", Algorithm 1): per-head
                    MSE against full attention, pattern sparsity, the loss
@@ -30,11 +34,14 @@ What it computes, and from where:
 Parity pins (``tests/test_oracle_*.py``): dense attention vs torch's float64
 ``scaled_dot_product_attention``; pooling vs ``avg_pool1d``; selection vs
 brute-force subset enumeration; patterns vs token-pair enumeration; the
-invariants of a convex combination; a hand-computable worked example.  The
+invariants of a convex combination; a hand-computable worked example; the
+gradients vs torch float64 autograd of SDPA and vs central finite differences
+of the forward oracle, with the softmax's shift and scaling identities.  The
 3D-tile pattern's block reading has only its own token-level definition to
 check against: its parity beyond that is unpinned.
 """
 from .asa import pool, pooled_probs, select_row, asa_mask, MaskInfo  # noqa: F401
 from .patterns import pattern_row, pattern_mask, keep_token_pair  # noqa: F401
 from .attention import masked_attention, attention_rows  # noqa: F401
+from .backward import attention_backward, mask_transpose  # noqa: F401
 from . import search  # noqa: F401
