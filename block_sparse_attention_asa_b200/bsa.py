@@ -48,6 +48,9 @@ _SIGNATURES = {
     "bsa_forward_workspace_size": (_c_size, [_c_int] * 5),
     "bsa_forward": (_c_int, [_vp, _vp, _vp] + [_c_int] * 5 + [_vp, _vp, _c_float, _vp, _vp, _vp,
                                                               _c_size, _vp]),
+    "bsa_backward_workspace_size": (_c_size, [_c_int] * 5),
+    "bsa_backward": (_c_int, [_vp] * 6 + [_c_int] * 5 + [_vp, _vp, _c_float, _vp, _vp, _vp, _vp,
+                                                          _c_size, _vp]),
     "bsa_check_device_status": (_c_int, [_vp]),
     "bsa_status_string": (ctypes.c_char_p, [_c_int]),
     "bsa_version": (_c_int, []),
@@ -253,6 +256,43 @@ def bsa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blk: int, row
         col_idx = torch.zeros(1, dtype=torch.int32, device=q.device)
     bsa_forward_into(q, k, v, blk, row_ptr, col_idx, o, lse, softmax_scale, ws, stream)
     return o, lse
+
+
+# ----------------------------------------------------------------------------- backward
+def backward_workspace_size(B: int, H: int, N: int, d: int, blk: int) -> int:
+    return int(load().bsa_backward_workspace_size(B, H, N, d, blk))
+
+
+def bsa_backward_into(q, k, v, o, dout, lse, blk, row_ptr, col_idx, dq, dk, dv,
+                      softmax_scale=0.0, workspace=None, stream=None):
+    B, H, N, d = _shape(q)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = load().bsa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), B, H, N,
+                             d, blk, _ptr(row_ptr), _ptr(col_idx), softmax_scale, _ptr(dq),
+                             _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "bsa_backward")
+
+
+def bsa_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                 dout: torch.Tensor, lse: torch.Tensor, blk: int, row_ptr: torch.Tensor,
+                 col_idx: torch.Tensor, softmax_scale: float = 0.0, stream=None):
+    """(dQ, dK, dV) bf16 [B,H,N,d] of attention over the CSR's kept blocks for the
+    incoming gradient dout; o and lse are bsa_forward's outputs for the same call."""
+    _need_cuda(q, k, v, o, dout, lse, row_ptr)
+    B, H, N, d = _shape(q)
+    for t in (k, v, o, dout):
+        if tuple(t.shape) != (B, H, N, d) or t.dtype != torch.bfloat16:
+            raise ValueError("k, v, o, dout must match q (bf16 [B, H, N, d])")
+    if lse.dtype != torch.float32 or tuple(lse.shape) != (B, H, N):
+        raise ValueError("lse must be float32 [B, H, N]")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(backward_workspace_size(B, H, N, d, blk), 256), dtype=torch.uint8,
+                     device=q.device)
+    if col_idx.numel() == 0:
+        col_idx = torch.zeros(1, dtype=torch.int32, device=q.device)
+    bsa_backward_into(q, k, v, o, dout, lse, blk, row_ptr, col_idx, dq, dk, dv, softmax_scale, ws,
+                      stream)
+    return dq, dk, dv
 
 
 def head_mse(o_ref: torch.Tensor, o: torch.Tensor, stream=None) -> torch.Tensor:

@@ -10,7 +10,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB = os.path.join(HERE, "libbsa_b200.so")
 SOURCES = [os.path.join(HERE, "csrc", "bsa_api.cu")]
 DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in
-                  ("common.cuh", "ptx.cuh", "pattern.cuh", "asa_mask.cuh", "bsa_fwd.cuh", "search.cuh")] + [
+                  ("common.cuh", "ptx.cuh", "pattern.cuh", "asa_mask.cuh", "bsa_fwd.cuh", "bsa_bwd.cuh", "search.cuh")] + [
     os.path.join(os.path.dirname(HERE), "include", "bsa.h")]
 
 NVCC_FLAGS = [

@@ -13,6 +13,7 @@
 #include "pattern.cuh"
 #include "asa_mask.cuh"
 #include "bsa_fwd.cuh"
+#include "bsa_bwd.cuh"
 #include "search.cuh"
 
 namespace {
@@ -286,6 +287,83 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
   return check_launch();
 }
 
+// ---- backward launches ---------------------------------------------------------
+// Raise a kernel's dynamic shared-memory limit once per device; `done` is the
+// caller's per-kernel flag array.
+template <typename KernelT>
+bool set_smem_once(KernelT kernel, int bytes, bool (&done)[64]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+template <int D, int BLK>
+int launch_bwd(const void* q, const void* k, const void* v, const void* dout, int B, int H,
+               int N, const int32_t* row_ptr, const int32_t* col_idx, const float* lse,
+               const float* delta, float scale, void* dq, void* dk, void* dv,
+               cudaStream_t stream) {
+  using C = bsa::BwdCfg<D, BLK>;
+  const int nb = (N + BLK - 1) / BLK;
+  const int nbw = (nb + 31) / 32;
+  if (nb > bsa::kBwdMaxNb || C::G * nbw * 4 > C::BM_BYTES) return BSA_ERR_UNSUPPORTED;
+  const int BH = B * H;
+  // resident tiles: 128-row boxes; gathered blocks: blk-row boxes
+  CUtensorMap q128, do128, k128, v128, qb, dob, kb, vb;
+  if (!make_map(&q128, q, BH, N, D, 128) || !make_map(&do128, dout, BH, N, D, 128) ||
+      !make_map(&k128, k, BH, N, D, 128) || !make_map(&v128, v, BH, N, D, 128) ||
+      !make_map(&qb, q, BH, N, D, BLK) || !make_map(&dob, dout, BH, N, D, BLK) ||
+      !make_map(&kb, k, BH, N, D, BLK) || !make_map(&vb, v, BH, N, D, BLK))
+    return BSA_ERR_CUDA;
+  static bool dq_set[64] = {}, dkdv_set[64] = {};
+  if (!set_smem_once(bsa::bsa_bwd_dq_kernel<D, BLK>, C::SMEM, dq_set) ||
+      !set_smem_once(bsa::bsa_bwd_dkdv_kernel<D, BLK>, C::SMEM, dkdv_set))
+    return BSA_ERR_CUDA;
+  bsa::BwdParams p;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.nb = nb;
+  p.nbw = nbw;
+  p.ntile = ceil_div(N, 128);
+  p.row_ptr = row_ptr;
+  p.col_idx = col_idx;
+  p.lse = lse;
+  p.delta = delta;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.wait_ns = kWaitNs;
+  const int items = BH * p.ntile;   // one 128-row tile per CTA, either side
+  bsa::bsa_bwd_dq_kernel<D, BLK><<<items, bsa::kBwdThreads, C::SMEM, stream>>>(q128, do128, kb,
+                                                                             vb, p);
+  if (check_launch()) return BSA_ERR_CUDA;
+  bsa::bsa_bwd_dkdv_kernel<D, BLK><<<items, bsa::kBwdThreads, C::SMEM, stream>>>(k128, v128, qb,
+                                                                               dob, p);
+  return check_launch();
+}
+
+template <int D>
+int launch_bwd_blk(int blk, const void* q, const void* k, const void* v, const void* dout, int B,
+                   int H, int N, const int32_t* rp, const int32_t* ci, const float* lse,
+                   const float* delta, float scale, void* dq, void* dk, void* dv,
+                   cudaStream_t s) {
+  switch (blk) {
+    case 16: return launch_bwd<D, 16>(q, k, v, dout, B, H, N, rp, ci, lse, delta, scale, dq, dk, dv, s);
+    case 32: return launch_bwd<D, 32>(q, k, v, dout, B, H, N, rp, ci, lse, delta, scale, dq, dk, dv, s);
+    case 64: return launch_bwd<D, 64>(q, k, v, dout, B, H, N, rp, ci, lse, delta, scale, dq, dk, dv, s);
+    case 128: return launch_bwd<D, 128>(q, k, v, dout, B, H, N, rp, ci, lse, delta, scale, dq, dk, dv, s);
+  }
+  return BSA_ERR_UNSUPPORTED;
+}
+
 }  // namespace
 
 extern "C" {
@@ -516,6 +594,47 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
   if (d == 64)
     return launch_fwd_blk<64>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);
   return launch_fwd_blk<128>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);
+}
+
+size_t bsa_backward_workspace_size(int B, int H, int N, int d, int blk) {
+  if (common_shape_checks(B, H, N, blk) != BSA_OK || (d != 64 && d != 128)) return 0;
+  return ((size_t)B * H * N * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+int bsa_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, int B, int H, int N, int d, int blk, const int32_t* row_ptr,
+                 const int32_t* col_idx, float softmax_scale, void* dq, void* dk, void* dv,
+                 void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !row_ptr || !col_idx || !dq || !dk || !dv)
+    return BSA_ERR_INVALID_ARG;
+  int rc = common_shape_checks(B, H, N, blk);
+  if (rc != BSA_OK) return rc;
+  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+      !aligned(lse, 4))
+    return BSA_ERR_UNSUPPORTED;
+  if ((N + blk - 1) / blk > bsa::kBwdMaxNb) return BSA_ERR_UNSUPPORTED;
+  if (std::isnan(softmax_scale)) return BSA_ERR_INVALID_ARG;
+  if (!workspace || ws_bytes < bsa_backward_workspace_size(B, H, N, d, blk) ||
+      !aligned(workspace, 256))
+    return BSA_ERR_WORKSPACE;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
+  cudaStream_t s = as_cuda(stream);
+  float* delta = static_cast<float*>(workspace);
+  const long long tokens = (long long)B * H * N;
+  const auto* ob = static_cast<const __nv_bfloat16*>(o);
+  const auto* db = static_cast<const __nv_bfloat16*>(dout);
+  if (d == 64) {
+    bsa::bwd_delta_kernel<64><<<ceil_div(tokens * 8, 256), 256, 0, s>>>(ob, db, tokens, delta);
+    if (check_launch()) return BSA_ERR_CUDA;
+    return launch_bwd_blk<64>(blk, q, k, v, dout, B, H, N, row_ptr, col_idx, lse, delta, scale,
+                              dq, dk, dv, s);
+  }
+  bsa::bwd_delta_kernel<128><<<ceil_div(tokens * 16, 256), 256, 0, s>>>(ob, db, tokens, delta);
+  if (check_launch()) return BSA_ERR_CUDA;
+  return launch_bwd_blk<128>(blk, q, k, v, dout, B, H, N, row_ptr, col_idx, lse, delta, scale,
+                             dq, dk, dv, s);
 }
 
 }  // extern "C"

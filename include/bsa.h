@@ -166,6 +166,33 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
                 float softmax_scale, void* o, float* lse,
                 void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
+/* ---- gradients of attention over kept blocks --------------------------------
+ * [BLADE] 技术框架: ASA is trained jointly with the step distillation, so the
+ * attention over the kept blocks is differentiated.  For a given dO (bf16
+ * [B,H,N,d]) this returns the gradient of the bsa_forward definition with
+ * respect to q, k and v, with the block mask held constant (its selection
+ * carries no gradient) and no gradient into lse:
+ *     P_tu = exp(scale q_t.k_u - lse_t)  over the listed key tokens u < N,
+ *     D_t = dO_t . O_t,   dS_tu = P_tu (dO_t . v_u - D_t),
+ *     dq_t = scale sum_u dS_tu k_u,  dk_u = scale sum_t dS_tu q_t,
+ *     dv_u = sum_t P_tu dO_t.
+ * o and lse are the outputs of bsa_forward on the same q, k, v, mask and
+ * scale (lse must not be NULL).  Each CSR row must be strictly ascending and
+ * nb must be at most 4096.  A token whose row lists nothing gets dq = 0 and
+ * adds nothing; a key token no row reaches gets dk = dv = 0.  Outputs dq, dk,
+ * dv are bf16 [B,H,N,d] (round to nearest even), each written once (no
+ * atomics: the result does not depend on scheduling); accumulation is fp32 on
+ * the tensor cores.  Workspace: bsa_backward_workspace_size() bytes, 256-byte
+ * aligned, holding D (fp32 [B,H,N]).  Asynchronous on `stream`.  A CSR block
+ * id outside [0, nb) is skipped and flagged (BSA_ERR_CSR in the device
+ * status). */
+size_t bsa_backward_workspace_size(int B, int H, int N, int d, int blk);
+int bsa_backward(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, int B, int H, int N, int d, int blk,
+                 const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale,
+                 void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                 bsa_stream_t stream);
+
 /* ---- Sparse-vDiT offline pattern search (diagnostic) ------------------------
  * Sparse-vDiT blog, "核心公式 / 离线搜索损失函数", "注意力模式选择" and
  * Algorithm 1: for each head and candidate pattern i,

@@ -133,3 +133,45 @@ def test_search_entry_points_validate_and_select_on_host(lib):
         ref_l = search.search_loss(mse, sp, lam)
         np.testing.assert_allclose(loss, ref_l, rtol=0, atol=0)
         assert choice.tolist() == search.select_pattern(ref_l, cand, eps).tolist()
+
+
+def test_backward_validation_and_workspace(lib):
+    vp = ctypes.c_void_p
+    # D (fp32 per token), rounded up to 256 bytes
+    assert bsa.backward_workspace_size(1, 12, 32760, 128, 64) == -(-12 * 32760 * 4 // 256) * 256
+    assert bsa.backward_workspace_size(1, 1, 10, 64, 16) == 256
+    assert lib.bsa_backward_workspace_size(1, 1, 100, 96, 16) == 0
+    args = [vp(256)] * 6 + [1, 1, 128, 64, 16, vp(256), vp(256), 0.0, vp(256), vp(256), vp(256),
+                            vp(256), 1 << 20, None]
+    for i in range(6):                       # q, k, v, o, dout, lse
+        bad = list(args)
+        bad[i] = None
+        assert lib.bsa_backward(*bad) == bsa.ERR_INVALID_ARG, i
+    for i in (11, 12, 14, 15, 16):           # row_ptr, col_idx, dq, dk, dv
+        bad = list(args)
+        bad[i] = None
+        assert lib.bsa_backward(*bad) == bsa.ERR_INVALID_ARG, i
+    bad = list(args)
+    bad[9] = 80                              # d
+    assert lib.bsa_backward(*bad) == bsa.ERR_UNSUPPORTED
+    bad = list(args)
+    bad[10] = 24                             # blk
+    assert lib.bsa_backward(*bad) == bsa.ERR_UNSUPPORTED
+    bad = list(args)
+    bad[4] = vp(264)                         # dout misaligned
+    assert lib.bsa_backward(*bad) == bsa.ERR_UNSUPPORTED
+    bad = list(args)
+    bad[8], bad[10] = 4097 * 16, 16          # nb over the backward's 4096
+    assert lib.bsa_backward(*bad) == bsa.ERR_UNSUPPORTED
+    bad = list(args)
+    bad[13] = float("nan")
+    assert lib.bsa_backward(*bad) == bsa.ERR_INVALID_ARG
+    bad = list(args)
+    bad[17] = None
+    assert lib.bsa_backward(*bad) == bsa.ERR_WORKSPACE
+    bad = list(args)
+    bad[18] = 16
+    assert lib.bsa_backward(*bad) == bsa.ERR_WORKSPACE
+    bad = list(args)
+    bad[17] = vp(272)
+    assert lib.bsa_backward(*bad) == bsa.ERR_WORKSPACE
