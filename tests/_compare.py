@@ -86,3 +86,53 @@ def compare_attention(o_gpu, lse_gpu, o_ref, lse_ref, rows_mask=None):
     assert rel_rms <= O_REL_RMS, f"O rel-RMS {rel_rms:.3e} > {O_REL_RMS}"
     assert lse_err <= LSE_ABS, f"LSE max-abs {lse_err:.3e} > {LSE_ABS}"
     return max_abs, rel_rms, lse_err
+
+
+# ---- gradients -----------------------------------------------------------------
+# dQ, dK, dV: rel-RMS <= 1e-2 and max|err| <= 2e-2 * max|ref| per gradient.  dQ
+# gets one more term: the kernel takes D_t = dO_t . Ô_t from the bf16 Ô the
+# forward returned, and an error dD_t in D moves dQ_t by scale * dD_t * k̄_t
+# (k̄_t = sum_u P_tu k_u, the attention of q over the keys with V := K).
+# Rounding O to bf16 has relative error at most u = 2^-8, independently per
+# element, so dD_t is within three standard deviations of a sum of uniform
+# terms: |dD_t| <= sqrt(3) * u * ||dO_t ∘ Ô_t||_2.  The dQ bounds add the RMS
+# (and the max) of scale * that * |k̄_t| to the base ones.
+GRAD_REL_RMS = 1e-2
+GRAD_MAX_REL = 2e-2
+BF16_U = 2.0 ** -8
+
+
+def d_term(do, o_hat, kbar, scale):
+    """Per-element size of the dQ error that D's rounding allows."""
+    do = np.asarray(do, dtype=np.float64)
+    o_hat = np.asarray(o_hat, dtype=np.float64)
+    dd = np.sqrt(3.0) * BF16_U * np.sqrt(np.sum((do * o_hat) ** 2, axis=-1))
+    return scale * dd[..., None] * np.abs(np.asarray(kbar, dtype=np.float64))
+
+
+def compare_gradients(got, ref, dq_term=None):
+    """got, ref: (dQ, dK, dV) arrays; dq_term: d_term(...) or None."""
+    out = []
+    for idx, (name, g, w) in enumerate(zip(("dq", "dk", "dv"), got, ref)):
+        g = np.asarray(g, dtype=np.float64)
+        w = np.asarray(w, dtype=np.float64)
+        assert np.all(np.isfinite(g)), f"{name}: non-finite"
+        err = np.abs(g - w)
+        wmax = float(np.abs(w).max()) if w.size else 0.0
+        wrms = float(np.sqrt(np.mean(w ** 2))) if w.size else 0.0
+        if wmax == 0.0:
+            assert float(err.max()) == 0.0, f"{name}: nonzero where the gradient is 0"
+            out.append((0.0, 0.0))
+            continue
+        extra_rms = extra_max = 0.0
+        if idx == 0 and dq_term is not None:
+            extra_rms = float(np.sqrt(np.mean(dq_term ** 2)))
+            extra_max = float(dq_term.max())
+        rms = float(np.sqrt(np.mean(err ** 2)))
+        mx = float(err.max())
+        assert rms <= GRAD_REL_RMS * wrms + extra_rms, \
+            f"{name}: RMS err {rms:.3e} > {GRAD_REL_RMS} * {wrms:.3e} + {extra_rms:.3e}"
+        assert mx <= GRAD_MAX_REL * wmax + extra_max, \
+            f"{name}: max err {mx:.3e} > {GRAD_MAX_REL} * {wmax:.3e} + {extra_max:.3e}"
+        out.append((rms / wrms, mx / wmax))
+    return out
