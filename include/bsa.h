@@ -26,11 +26,13 @@
  *    wait that gave up) are recorded in a per-device status word read by
  *    bsa_check_device_status().  No C++ exception crosses this interface.
  *  - Supported: d in {64, 128}; blk in {16, 32, 64, 128}; N >= 1; B, H >= 1;
- *    B*H*nb*nb < 2^31.  The device must be sm_100 (B200).
+ *    B*H*nb*nb < 2^31 (the backward also nb <= 4096).  The device must be
+ *    sm_100 (B200).
  *
  * Sources (web pages on the method):
  *  [BLADE]   "BLADE: Block-Sparse Attention Meets Step Distillation for
- *            Efficient Video Generation" (digest: abstract; 方法详解 / 关键设计)
+ *            Efficient Video Generation" (digest: abstract; 技术框架;
+ *            方法详解 / 关键设计)
  *  [SvDiT]   "Sparse-vDiT: Sparse Attention Acceleration for Video Diffusion
  *            Transformers" (blog: 核心公式; 四种注意力模式 table; 模型组件)
  *  [EvDiT]   "Efficient-vDiT: Efficient Video Diffusion Transformers With
