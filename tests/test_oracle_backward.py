@@ -13,7 +13,10 @@
 * special cases: skip rows get dQ = 0 and feed nothing; one block of identical
   keys gives dQ = 0 and dV = the mean of dO over its queries; a permutation
   inside a kept block permutes dK and dV and leaves dQ;
-* the transpose vs a dense boolean block matrix, and transposing twice.
+* the transpose vs a dense boolean block matrix, and transposing twice;
+* the GPU tests' gradient bounds accept the oracle's own result and reject
+  planted mistakes (a dropped scale, swapped gradients, another scale, another
+  mask).
 """
 import math
 
@@ -215,3 +218,28 @@ def test_mask_transpose_vs_dense(seed):
     # the transpose of the transpose is the mask
     rp2, ci2 = oracle.mask_transpose(cp, ri, B, H, nb)
     assert np.array_equal(rp2, rp) and np.array_equal(ci2, ci)
+
+
+def test_gradient_comparator_rejects_planted_mistakes():
+    # the GPU tests' bounds (tests/_compare.py) accept the oracle and reject
+    # a dropped scale, swapped gradients, another softmax scale and another mask
+    from tests._compare import compare_gradients, d_term
+    B, H, N, d, blk = 1, 2, 96, 64, 16
+    nb = N // blk
+    q, k, v, do = _qkv(B, H, N, d, 17)
+    rp, ci, _ = _random_csr(B * H * nb, nb, 5, p_empty=0.2)
+    ref = oracle.attention_backward(q, k, v, do, blk, rp, ci)
+    o, lse = oracle.masked_attention(q, k, v, blk, rp, ci)
+    kbar, _ = oracle.masked_attention(q, k, k, blk, rp, ci)
+    term = d_term(do, o, kbar, 1 / math.sqrt(d))
+    compare_gradients(ref, ref, term)
+    bad = [
+        (ref[0] * math.sqrt(d), ref[1], ref[2]),                       # dQ without the scale
+        (ref[0], ref[2], ref[1]),                                      # dK and dV swapped
+        oracle.attention_backward(q, k, v, do, blk, rp, ci, 0.2),      # another scale
+    ]
+    rp2, ci2, _ = _random_csr(B * H * nb, nb, 6, p_empty=0.2)
+    bad.append(oracle.attention_backward(q, k, v, do, blk, rp2, ci2))  # another mask
+    for g in bad:
+        with pytest.raises(AssertionError):
+            compare_gradients(g, ref, term)
