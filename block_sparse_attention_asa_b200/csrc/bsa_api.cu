@@ -615,6 +615,8 @@ int bsa_backward(const void* q, const void* k, const void* v, const void* o, con
       !aligned(lse, 4))
     return BSA_ERR_UNSUPPORTED;
   if ((N + blk - 1) / blk > bsa::kBwdMaxNb) return BSA_ERR_UNSUPPORTED;
+  // the D pass runs d/8 threads per token in a 1D grid of 256-thread blocks
+  if ((long long)B * H * N * (d / 8) > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
   if (std::isnan(softmax_scale)) return BSA_ERR_INVALID_ARG;
   if (!workspace || ws_bytes < bsa_backward_workspace_size(B, H, N, d, blk) ||
       !aligned(workspace, 256))

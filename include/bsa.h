@@ -179,8 +179,8 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
  *     dq_t = scale sum_u dS_tu k_u,  dk_u = scale sum_t dS_tu q_t,
  *     dv_u = sum_t P_tu dO_t.
  * o and lse are the outputs of bsa_forward on the same q, k, v, mask and
- * scale (lse must not be NULL).  Each CSR row must be strictly ascending and
- * nb must be at most 4096.  A token whose row lists nothing gets dq = 0 and
+ * scale (lse must not be NULL).  Each CSR row must be strictly ascending,
+ * nb must be at most 4096 and B*H*N*d/8 below 2^31.  A token whose row lists nothing gets dq = 0 and
  * adds nothing; a key token no row reaches gets dk = dv = 0.  Outputs dq, dk,
  * dv are bf16 [B,H,N,d] (round to nearest even), each written once (no
  * atomics: the result does not depend on scheduling); accumulation is fp32 on

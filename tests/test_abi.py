@@ -164,6 +164,9 @@ def test_backward_validation_and_workspace(lib):
     bad[8], bad[10] = 4097 * 16, 16          # nb over the backward's 4096
     assert lib.bsa_backward(*bad) == bsa.ERR_UNSUPPORTED
     bad = list(args)
+    bad[6], bad[7], bad[8], bad[9], bad[10] = 65535, 1, 4096, 128, 128   # B*H*N*d/8 past 2^31
+    assert lib.bsa_backward(*bad) == bsa.ERR_UNSUPPORTED
+    bad = list(args)
     bad[13] = float("nan")
     assert lib.bsa_backward(*bad) == bsa.ERR_INVALID_ARG
     bad = list(args)
