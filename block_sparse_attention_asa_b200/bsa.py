@@ -55,6 +55,7 @@ _SIGNATURES = {
     "bsa_status_string": (ctypes.c_char_p, [_c_int]),
     "bsa_version": (_c_int, []),
     "bsa_debug_exp2_poly": (_c_int, [_vp, _vp, _c_int, _vp]),
+    "bsa_debug_wait_timeout": (_c_int, [ctypes.c_ulonglong, _c_int, _vp, _vp]),
     "attention_head_mse_workspace_size": (_c_size, [_c_int] * 4),
     "attention_head_mse": (_c_int, [_vp, _vp] + [_c_int] * 4 + [_vp, _vp, _c_size, _vp]),
     "csr_head_sparsity_workspace_size": (_c_size, [_c_int]),
@@ -345,6 +346,19 @@ def debug_exp2_poly(x: torch.Tensor, stream=None) -> torch.Tensor:
     _check(load().bsa_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)),
            "bsa_debug_exp2_poly")
     return y
+
+
+def debug_wait_timeout(limit_ns: int, arrive_first: bool = False,
+                       waited: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Run the library's bounded mbarrier wait on a phase that completes only if
+    arrive_first; without it the wait gives up after limit_ns and the device
+    status reads ERR_TIMEOUT.  waited: optional CUDA int64 [1], the time taken."""
+    if waited is not None:
+        _need_cuda(waited)
+        if waited.dtype != torch.int64 or waited.numel() < 1:
+            raise ValueError("waited must be a CUDA int64 tensor")
+    _check(load().bsa_debug_wait_timeout(int(limit_ns), int(bool(arrive_first)), _ptr(waited),
+                                         _stream(stream)), "bsa_debug_wait_timeout")
 
 
 def default_scale(d: int) -> float:

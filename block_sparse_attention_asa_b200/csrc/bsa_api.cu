@@ -648,6 +648,33 @@ __global__ void exp2_poly_kernel(const float* x, float* y, int n) {
 }
 }  // namespace
 
+namespace {
+// One thread waits, with the bounded wait every kernel of this library uses,
+// on an mbarrier phase that completes only if the thread arrives first.
+// Without the arrive the wait gives up after limit_ns, the kernel records
+// BSA_ERR_TIMEOUT and returns.
+__global__ void wait_timeout_kernel(unsigned long long limit_ns, int arrive_first,
+                                    unsigned long long* waited_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  bsa::mbar_init(&bar, 1);
+  bsa::fence_mbar_init();
+  if (arrive_first) bsa::mbar_arrive(&bar);
+  const uint64_t t0 = bsa::global_ns();
+  const bool ok = bsa::mbar_wait(&bar, 0, limit_ns);
+  if (waited_ns) *waited_ns = bsa::global_ns() - t0;
+  if (!ok) bsa::record_error(BSA_ERR_TIMEOUT);
+}
+}  // namespace
+
+extern "C" int bsa_debug_wait_timeout(unsigned long long limit_ns, int arrive_first,
+                                      unsigned long long* waited_ns, bsa_stream_t stream) {
+  if (limit_ns > 10000000000ull) return BSA_ERR_INVALID_ARG;   // at most 10 s
+  if (waited_ns && !aligned(waited_ns, 8)) return BSA_ERR_UNSUPPORTED;
+  wait_timeout_kernel<<<1, 32, 0, as_cuda(stream)>>>(limit_ns, arrive_first, waited_ns);
+  return check_launch();
+}
+
 extern "C" int bsa_debug_exp2_poly(const float* x, float* y, int n, bsa_stream_t stream) {
   if (!x || !y || n < 0) return BSA_ERR_INVALID_ARG;
   if (n == 0) return BSA_OK;

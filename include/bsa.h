@@ -241,6 +241,16 @@ const char* bsa_status_string(int status);
  * pointers, n floats; asynchronous on `stream`.  For testing the kernel's
  * arithmetic against the CUDA math library; no counterpart on the pages. */
 int bsa_debug_exp2_poly(const float* x, float* y, int n, bsa_stream_t stream);
+/* Diagnostics: failure detection without a GPU fault.  One thread waits, with
+ * the bounded wait that every kernel of this library uses on its mbarriers,
+ * on a phase that completes only when arrive_first is nonzero.  Without the
+ * arrive the wait gives up after limit_ns nanoseconds (at most 10 s, else
+ * BSA_ERR_INVALID_ARG), BSA_ERR_TIMEOUT is recorded in the device status and
+ * the kernel returns: the context stays usable.  waited_ns (device, 8-byte
+ * aligned, may be NULL) receives how long the wait took.  Asynchronous on
+ * `stream`.  No counterpart on the pages. */
+int bsa_debug_wait_timeout(unsigned long long limit_ns, int arrive_first,
+                           unsigned long long* waited_ns, bsa_stream_t stream);
 /* Library version as major*10000 + minor*100 + patch. */
 int bsa_version(void);
 

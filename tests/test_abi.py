@@ -178,3 +178,9 @@ def test_backward_validation_and_workspace(lib):
     bad = list(args)
     bad[17] = vp(272)
     assert lib.bsa_backward(*bad) == bsa.ERR_WORKSPACE
+
+
+def test_wait_timeout_diagnostic_validation(lib):
+    vp = ctypes.c_void_p
+    assert lib.bsa_debug_wait_timeout(10_000_000_001, 0, None, None) == bsa.ERR_INVALID_ARG
+    assert lib.bsa_debug_wait_timeout(1000, 0, vp(260), None) == bsa.ERR_UNSUPPORTED
