@@ -51,6 +51,7 @@ _SIGNATURES = {
     "bsa_backward_workspace_size": (_c_size, [_c_int] * 5),
     "bsa_backward": (_c_int, [_vp] * 6 + [_c_int] * 5 + [_vp, _vp, _c_float, _vp, _vp, _vp, _vp,
                                                           _c_size, _vp]),
+    "bsa_validate_csr_host": (_c_int, [_vp, _vp, _c_i64, _c_int, _c_i64, _vp]),
     "bsa_check_device_status": (_c_int, [_vp]),
     "bsa_status_string": (ctypes.c_char_p, [_c_int]),
     "bsa_version": (_c_int, []),
@@ -128,6 +129,20 @@ def _shape(q: torch.Tensor):
     if q.dim() != 4 or q.dtype != torch.bfloat16:
         raise ValueError("q/k/v must be bf16 [B, H, N, d]")
     return tuple(int(x) for x in q.shape)
+
+
+def validate_csr(row_ptr, col_idx, nb: int) -> int:
+    """-1 if the CSR block mask (host arrays or tensors) follows the library's
+    conventions (rows strictly ascending, ids in [0, nb)), else the first bad row."""
+    import numpy as np
+    rp = np.ascontiguousarray(torch.as_tensor(row_ptr).cpu().numpy(), dtype=np.int32)
+    ci = np.ascontiguousarray(torch.as_tensor(col_idx).cpu().numpy(), dtype=np.int32)
+    bad = ctypes.c_int64(-1)
+    rc = load().bsa_validate_csr_host(rp.ctypes.data, ci.ctypes.data if ci.size else None,
+                                      len(rp) - 1, int(nb), ci.size, ctypes.byref(bad))
+    if rc not in (OK, ERR_CSR):
+        _check(rc, "bsa_validate_csr_host")
+    return int(bad.value)
 
 
 def check_device_status(stream=None) -> int:

@@ -461,6 +461,28 @@ int pattern_search_select(const double* mse, const double* sparsity, const int32
   return BSA_OK;
 }
 
+int bsa_validate_csr_host(const int32_t* row_ptr_host, const int32_t* col_idx_host, int64_t rows,
+                          int nb, int64_t col_len, int64_t* bad_row_host) {
+  if (!row_ptr_host || rows < 0 || nb <= 0 || col_len < 0 || (!col_idx_host && col_len > 0))
+    return BSA_ERR_INVALID_ARG;
+  auto fail = [&](int64_t r) {
+    if (bad_row_host) *bad_row_host = r;
+    return BSA_ERR_CSR;
+  };
+  if (row_ptr_host[0] != 0) return fail(0);
+  for (int64_t r = 0; r < rows; ++r) {
+    const int64_t e0 = row_ptr_host[r], e1 = row_ptr_host[r + 1];
+    if (e1 < e0 || e1 > col_len) return fail(r);
+    for (int64_t e = e0; e < e1; ++e) {
+      const int32_t c = col_idx_host[e];
+      if (c < 0 || c >= nb) return fail(r);
+      if (e > e0 && col_idx_host[e - 1] >= c) return fail(r);
+    }
+  }
+  if (bad_row_host) *bad_row_host = -1;
+  return BSA_OK;
+}
+
 int bsa_check_device_status(bsa_stream_t stream) {
   if (cudaStreamSynchronize(as_cuda(stream)) != cudaSuccess) return BSA_ERR_CUDA;
   int v = 0;

@@ -228,6 +228,16 @@ int csr_head_sparsity(const int32_t* row_ptr, const int32_t* col_idx, int B, int
 int pattern_search_select(const double* mse, const double* sparsity, const int32_t* candidates,
                           int P, int H, double lambda, double eps, double* loss, int32_t* choice);
 
+/* ---- CSR check (host) ---------------------------------------------------------
+ * bsa_validate_csr_host checks a block mask held in HOST memory against the
+ * conventions above: row_ptr[0] = 0, non-decreasing, row_ptr[rows] <= col_len
+ * (the length of col_idx_host), every block id in [0, nb) and each row strictly
+ * ascending (as bsa_backward requires; bsa_forward tolerates any order).
+ * Returns BSA_OK, or BSA_ERR_CSR with the first offending row in
+ * *bad_row_host (may be NULL; -1 when the mask is valid).  No device work. */
+int bsa_validate_csr_host(const int32_t* row_ptr_host, const int32_t* col_idx_host, int64_t rows,
+                          int nb, int64_t col_len, int64_t* bad_row_host);
+
 /* ---- status ----------------------------------------------------------------
  * bsa_check_device_status synchronizes `stream`, returns the first error any
  * kernel of this library recorded on the current device since the last check

@@ -184,3 +184,40 @@ def test_wait_timeout_diagnostic_validation(lib):
     vp = ctypes.c_void_p
     assert lib.bsa_debug_wait_timeout(10_000_000_001, 0, None, None) == bsa.ERR_INVALID_ARG
     assert lib.bsa_debug_wait_timeout(1000, 0, vp(260), None) == bsa.ERR_UNSUPPORTED
+
+
+def test_host_csr_validator(lib):
+    import numpy as np
+    # valid: empty row, full row, ragged
+    rp = np.array([0, 0, 3, 5], dtype=np.int32)
+    ci = np.array([0, 1, 2, 1, 2], dtype=np.int32)
+    assert bsa.validate_csr(rp, ci, 3) == -1
+    assert bsa.validate_csr(np.zeros(4, dtype=np.int32), np.zeros(0, dtype=np.int32), 3) == -1
+    bad_cases = [
+        (np.array([1, 1, 3, 5]), ci, 0),                 # row_ptr[0] != 0
+        (np.array([0, 3, 2, 5]), ci, 1),                 # decreasing row_ptr
+        (np.array([0, 0, 3, 6]), ci, 2),                 # past the end of col_idx
+        (rp, np.array([0, 1, 3, 1, 2]), 1),              # id >= nb
+        (rp, np.array([0, 1, 2, -1, 2]), 2),             # negative id
+        (rp, np.array([0, 2, 1, 1, 2]), 1),              # descending inside a row
+        (rp, np.array([0, 1, 2, 2, 2]), 2),              # duplicate
+    ]
+    for rpb, cib, row in bad_cases:
+        assert bsa.validate_csr(np.asarray(rpb, np.int32), np.asarray(cib, np.int32), 3) == row
+    vp = ctypes.c_void_p
+    assert lib.bsa_validate_csr_host(None, None, 1, 3, 0, None) == bsa.ERR_INVALID_ARG
+    assert lib.bsa_validate_csr_host(vp(16), None, 1, 3, 5, None) == bsa.ERR_INVALID_ARG
+
+
+def test_oracle_masks_pass_the_validator(lib):
+    # the oracle's ASA and pattern masks follow the conventions the kernels rely on
+    import numpy as np
+    import oracle
+    from block_sparse_attention_asa_b200 import workloads as W
+    w = W.TINY
+    q, k, _ = W.make_qkv(w)
+    info = oracle.asa_mask(W.as_f64(q), W.as_f64(k), w.blk, w.mode, w.topk, w.mass_tau,
+                           w.max_keep_ratio, w.keep_diag, w.n_sink_blocks)
+    assert bsa.validate_csr(info.row_ptr.astype(np.int32), info.col_idx, w.nb) == -1
+    rp, ci = oracle.pattern_mask([0, 1, 2, 3, 4, 5], 1, 6, 300, 16, 2, 64, -1, 1, 1, 1)
+    assert bsa.validate_csr(np.asarray(rp, np.int32), np.asarray(ci, np.int32), 19) == -1
