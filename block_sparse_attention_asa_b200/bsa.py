@@ -311,6 +311,36 @@ def bsa_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Ten
     return dq, dk, dv
 
 
+class _BlockSparseAttention(torch.autograd.Function):
+    """bsa_forward / bsa_backward as one autograd node.  The mask is a constant
+    of the step and only O is returned, so nothing downstream can depend on an
+    undifferentiated LSE."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, blk, row_ptr, col_idx, softmax_scale):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, lse = bsa_forward(q, k, v, blk, row_ptr, col_idx, softmax_scale)
+        ctx.save_for_backward(q, k, v, o, lse, row_ptr, col_idx)
+        ctx.blk = blk
+        ctx.softmax_scale = softmax_scale
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, lse, row_ptr, col_idx = ctx.saved_tensors
+        dq, dk, dv = bsa_backward(q, k, v, o, dout.contiguous().to(torch.bfloat16), lse, ctx.blk,
+                                  row_ptr, col_idx, ctx.softmax_scale)
+        return dq, dk, dv, None, None, None, None
+
+
+def block_sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blk: int,
+                           row_ptr: torch.Tensor, col_idx: torch.Tensor,
+                           softmax_scale: float = 0.0) -> torch.Tensor:
+    """Differentiable O of attention over the CSR's kept blocks (bf16 [B,H,N,d]);
+    gradients flow to q, k and v, none to the mask."""
+    return _BlockSparseAttention.apply(q, k, v, blk, row_ptr, col_idx, softmax_scale)
+
+
 def head_mse(o_ref: torch.Tensor, o: torch.Tensor, stream=None) -> torch.Tensor:
     """Per-head MSE(O - O_ref) over all B*N*d elements, float64 [H] on the device."""
     _need_cuda(o_ref, o)

@@ -9,7 +9,8 @@ the kernel's arithmetic (P and dS rounded to bf16 before their products, D
 from the bf16 O, fp32 sums, bf16 outputs) lands at about 2.4e-3 rel-RMS and
 5e-3 max on these cases.  Tokens whose row lists nothing get dQ exactly 0; key
 tokens no row reaches get dK and dV exactly 0.  Two runs give identical bits
-(no atomics).
+(no atomics).  The autograd node of the binding (block_sparse_attention)
+returns exactly the kernels' O and gradients.
 """
 import numpy as np
 import pytest
@@ -122,3 +123,21 @@ def test_backward_is_deterministic(cuda_lib):
     assert cuda_lib.check_device_status() == 0
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+def test_autograd_node_returns_the_kernels_gradients(cuda_lib):
+    B, H, N, d, blk = 1, 2, 300, 64, 64
+    nb = -(-N // blk)
+    rp, ci, _ = _csr(B * H * nb, nb, 41)
+    g = torch.Generator().manual_seed(9)
+    q, k, v, do = (torch.randn(B, H, N, d, generator=g).to(torch.bfloat16).cuda() for _ in range(4))
+    rpd, cid = torch.as_tensor(rp).cuda(), torch.as_tensor(ci).cuda()
+    qa, ka, va = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o = cuda_lib.block_sparse_attention(qa, ka, va, blk, rpd, cid)
+    o.backward(do)
+    o2, lse = cuda_lib.bsa_forward(q, k, v, blk, rpd, cid)
+    dq, dk, dv = cuda_lib.bsa_backward(q, k, v, o2, do, lse, blk, rpd, cid)
+    assert cuda_lib.check_device_status() == 0
+    assert torch.equal(o.detach(), o2)
+    for got, want in ((qa.grad, dq), (ka.grad, dk), (va.grad, dv)):
+        assert got.dtype == torch.bfloat16 and torch.equal(got, want)
