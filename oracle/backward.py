@@ -91,3 +91,68 @@ def mask_transpose(row_ptr, col_idx, B: int, H: int, nb: int):
     col_ptr[1:] = np.cumsum([len(c) for c in cols])
     row_idx = np.asarray([i for c in cols for i in sorted(c)], dtype=np.int32)
     return col_ptr, row_idx
+
+
+def attention_backward_sampled(q, k, v, do, blk: int, row_ptr, col_idx, q_rows, kv_cols,
+                               scale: float | None = None):
+    """The same gradients, for a sample only.
+
+    q_rows: CSR row ids r = (b*H + h)*nb + i -> {r: dQ [tokens of q-block i, d]}.
+    kv_cols: ids c = (b*H + h)*nb + j -> {c: (dK, dV) [tokens of kv-block j, d]},
+    summed over every row of that (b, h) that lists j.
+    """
+    q, k, v, do = (np.asarray(x) for x in (q, k, v, do))
+    B, H, n, d = q.shape
+    nb = -(-n // blk)
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    col_idx = np.asarray(col_idx, dtype=np.int64)
+
+    def row_terms(r):
+        i = r % nb
+        bh = r // nb
+        b, h = bh // H, bh % H
+        t0, t1 = i * blk, min(n, (i + 1) * blk)
+        cols = col_idx[row_ptr[r]:row_ptr[r + 1]]
+        keys = _row_keys(cols, blk, n)
+        qt = q[b, h, t0:t1].astype(np.float64)
+        dot = do[b, h, t0:t1].astype(np.float64)
+        kt = k[b, h, keys].astype(np.float64)
+        vt = v[b, h, keys].astype(np.float64)
+        s = (qt @ kt.T) * scale
+        e = np.exp(s - s.max(axis=1, keepdims=True))
+        p = e / e.sum(axis=1, keepdims=True)
+        dp = dot @ vt.T
+        ds = p * (dp - (p * dp).sum(axis=1, keepdims=True))
+        return keys, qt, dot, kt, p, ds
+
+    dq = {}
+    for r in q_rows:
+        r = int(r)
+        i = r % nb
+        rows_here = min(n, (i + 1) * blk) - i * blk
+        if row_ptr[r + 1] == row_ptr[r]:
+            dq[r] = np.zeros((rows_here, d))
+            continue
+        keys, qt, dot, kt, p, ds = row_terms(r)
+        dq[r] = scale * (ds @ kt)
+    dkv = {}
+    for c in kv_cols:
+        c = int(c)
+        j = c % nb
+        bh = c // nb
+        u0, u1 = j * blk, min(n, (j + 1) * blk)
+        gk = np.zeros((u1 - u0, d))
+        gv = np.zeros((u1 - u0, d))
+        for i in range(nb):
+            r = bh * nb + i
+            cols = col_idx[row_ptr[r]:row_ptr[r + 1]]
+            if j not in cols:
+                continue
+            keys, qt, dot, kt, p, ds = row_terms(r)
+            sel = (keys >= u0) & (keys < u1)
+            gv += p[:, sel].T @ dot
+            gk += scale * (ds[:, sel].T @ qt)
+        dkv[c] = (gk, gv)
+    return dq, dkv

@@ -243,3 +243,21 @@ def test_gradient_comparator_rejects_planted_mistakes():
     for g in bad:
         with pytest.raises(AssertionError):
             compare_gradients(g, ref, term)
+
+
+def test_sampled_gradients_equal_the_full_ones():
+    # the per-row / per-kv-block restatement used at full layer sizes
+    B, H, N, d, blk = 2, 2, 90, 64, 16
+    nb = -(-N // blk)
+    q, k, v, do = _qkv(B, H, N, d, 23)
+    rp, ci, _ = _random_csr(B * H * nb, nb, 4, p_empty=0.2)
+    full = oracle.attention_backward(q, k, v, do, blk, rp, ci)
+    rows = range(B * H * nb)
+    dq, dkv = oracle.attention_backward_sampled(q, k, v, do, blk, rp, ci, rows, rows)
+    for r in rows:
+        bh, i = divmod(r, nb)
+        b, h = divmod(bh, H)
+        t = slice(i * blk, min(N, (i + 1) * blk))
+        np.testing.assert_allclose(dq[r], full[0][b, h, t], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dkv[r][0], full[1][b, h, t], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dkv[r][1], full[2][b, h, t], rtol=0, atol=1e-12)
