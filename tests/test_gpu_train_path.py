@@ -1,0 +1,84 @@
+"""The training path end to end, through the C ABI: the binding's autograd node
+and the backward on the bench's full layers.
+
+* block_sparse_attention (one autograd node over bsa_forward / bsa_backward)
+  returns exactly the kernels' O and gradients;
+* on the Wan and Cog layers (GPU mask -> forward -> backward), 16 random
+  q-blocks plus the last (dQ) and 16 random kv-blocks plus the first and last
+  (dK, dV) match the oracle's per-block restatement
+  (oracle.attention_backward_sampled) within the gradient bounds of
+  tests/_compare.py, the dQ term for the rounding of O included.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_sparse_attention_asa_b200 import workloads as W
+from tests._compare import compare_gradients, d_term
+from tests.test_gpu_backward import _csr
+
+pytestmark = pytest.mark.gpu
+
+
+def test_autograd_node_returns_the_kernels_gradients(cuda_lib):
+    B, H, N, d, blk = 1, 2, 300, 64, 64
+    nb = -(-N // blk)
+    rp, ci, _ = _csr(B * H * nb, nb, 41)
+    g = torch.Generator().manual_seed(9)
+    q, k, v, do = (torch.randn(B, H, N, d, generator=g).to(torch.bfloat16).cuda() for _ in range(4))
+    rpd, cid = torch.as_tensor(rp).cuda(), torch.as_tensor(ci).cuda()
+    qa, ka, va = (t.clone().requires_grad_(True) for t in (q, k, v))
+    o = cuda_lib.block_sparse_attention(qa, ka, va, blk, rpd, cid)
+    o.backward(do)
+    o2, lse = cuda_lib.bsa_forward(q, k, v, blk, rpd, cid)
+    dq, dk, dv = cuda_lib.bsa_backward(q, k, v, o2, do, lse, blk, rpd, cid)
+    assert cuda_lib.check_device_status() == 0
+    assert torch.equal(o.detach(), o2)
+    for got, want in ((qa.grad, dq), (ka.grad, dk), (va.grad, dv)):
+        assert got.dtype == torch.bfloat16 and torch.equal(got, want)
+
+
+@pytest.mark.parametrize("w", [W.WAN, W.COG], ids=lambda w: w.name)
+def test_backward_full_config_sampled(cuda_lib, w):
+    # the bench's layers end to end (GPU mask -> forward -> backward), checked
+    # on 16+ sampled q-blocks (dQ) and 16+ sampled kv-blocks (dK, dV)
+    q, k, v = W.make_qkv(w)
+    g = torch.Generator().manual_seed(77)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    rp, ci = cuda_lib.asa_build_mask(qd, kd, w.blk, w.mode, w.topk, w.mass_tau, w.max_keep_ratio,
+                                     w.keep_diag, w.n_sink_blocks)
+    o, lse = cuda_lib.bsa_forward(qd, kd, vd, w.blk, rp, ci)
+    dq, dk, dv = cuda_lib.bsa_backward(qd, kd, vd, o, dod, lse, w.blk, rp, ci)
+    assert cuda_lib.check_device_status() == 0
+    B, H, N, d = q.shape
+    nb, blk = w.nb, w.blk
+    rp_h, ci_h = rp.cpu().numpy().astype(np.int64), ci.cpu().numpy()
+    rng = np.random.default_rng(19)
+    rows = sorted(set(rng.choice(B * H * nb, size=16, replace=False).tolist() + [nb - 1]))
+    cols = sorted(set(rng.choice(B * H * nb, size=16, replace=False).tolist() + [0, nb - 1]))
+    qf, kf, vf, dof = W.as_f64(q), W.as_f64(k), W.as_f64(v), W.as_f64(do)
+    ref_dq, ref_dkv = oracle.attention_backward_sampled(qf, kf, vf, dof, blk, rp_h, ci_h, rows,
+                                                        cols)
+    kbar = oracle.attention_rows(qf, kf, kf, blk, rp_h, ci_h, rows)
+    dqh, dkh, dvh = (x.float().cpu().numpy() for x in (dq, dk, dv))
+    oh = o.float().cpu().numpy()
+    got, ref, term = ([], [], []), ([], [], []), []
+    for r in rows:
+        bh, i = divmod(r, nb)
+        b, h = divmod(bh, H)
+        t = slice(i * blk, min(N, (i + 1) * blk))
+        got[0].append(dqh[b, h, t])
+        ref[0].append(ref_dq[r])
+        term.append(d_term(dof[b, h, t], oh[b, h, t], kbar[r][0], 1.0 / np.sqrt(d)))
+    for c in cols:
+        bh, j = divmod(c, nb)
+        b, h = divmod(bh, H)
+        t = slice(j * blk, min(N, (j + 1) * blk))
+        got[1].append(dkh[b, h, t])
+        got[2].append(dvh[b, h, t])
+        ref[1].append(ref_dkv[c][0])
+        ref[2].append(ref_dkv[c][1])
+    compare_gradients([np.concatenate(x) for x in got], [np.concatenate(x) for x in ref],
+                      np.concatenate(term))
