@@ -4,6 +4,8 @@
 * softmax  vs torch.softmax (library routine) on the pooled scores
 * top-k / mass selection vs brute-force enumeration of every subset (nb = 8)
 * the hand-computable worked example (tests/golden/worked_example.json)
+* degenerate cases: tau = 1 and k >= nb keep every block, a head of one
+  block keeps it, a single-token layer gives O = v and LSE = q.k * scale
 """
 import itertools
 import json
@@ -149,3 +151,30 @@ def test_worked_example_attention():
     np.testing.assert_allclose(o[0, 0, ::2, 0], g["full"]["O_per_block"], atol=g["tol"])
     assert lse[0, 0, 2] == pytest.approx(g["full"]["LSE_row1"], abs=g["tol"])
     assert lse[0, 0, 2] == pytest.approx(math.log(8), abs=1e-15)
+
+
+def test_degenerate_selections():
+    rng = np.random.default_rng(4)
+    for _ in range(20):
+        p = rng.dirichlet(np.ones(8))
+        # tau = 1 needs every block, also when the probabilities sum to just under 1
+        assert oracle.select_row(p, 0, MODE_MASS, mass_tau=1.0).cols == list(range(8))
+        # k at or above nb keeps every block
+        for k in (8, 9, 100):
+            assert oracle.select_row(p, 3, MODE_TOPK, topk=k).cols == list(range(8))
+    # a single block per head (N <= blk): the only block, whatever the rule
+    q, k = _rand((1, 2, 5, 4), 1), _rand((1, 2, 5, 4), 2)
+    for mode, kw in ((MODE_TOPK, dict(topk=3)), (MODE_MASS, dict(mass_tau=0.5))):
+        m = oracle.asa_mask(q, k, 16, mode, **kw)
+        assert m.row_ptr.tolist() == [0, 1, 2] and m.col_idx.tolist() == [0, 0]
+
+
+def test_single_token_layer():
+    # N = 1: the pooled block is the token, the mask keeps it, O = v and
+    # LSE = q.k * scale (one key: softmax weight 1)
+    q, k, v = _rand((1, 1, 1, 4), 5), _rand((1, 1, 1, 4), 6), _rand((1, 1, 1, 4), 7)
+    np.testing.assert_array_equal(oracle.pool(q, 16), q)
+    m = oracle.asa_mask(q, k, 16, MODE_TOPK, topk=1)
+    o, lse = oracle.masked_attention(q, k, v, 16, m.row_ptr, m.col_idx)
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-15)
+    assert abs(lse[0, 0, 0] - float((q * k).sum()) / 2.0) < 1e-15
