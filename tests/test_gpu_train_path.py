@@ -7,7 +7,9 @@ and the backward on the bench's full layers.
   q-blocks plus the last (dQ) and 16 random kv-blocks plus the first and last
   (dK, dV) match the oracle's per-block restatement
   (oracle.attention_backward_sampled) within the gradient bounds of
-  tests/_compare.py, the dQ term for the rounding of O included.
+  tests/_compare.py, the dQ term for the rounding of O included;
+* sequences of 1 to 17 tokens (one partial block per head) through mask,
+  forward and backward.
 """
 import numpy as np
 import pytest
@@ -82,3 +84,28 @@ def test_backward_full_config_sampled(cuda_lib, w):
         ref[2].append(ref_dkv[c][1])
     compare_gradients([np.concatenate(x) for x in got], [np.concatenate(x) for x in ref],
                       np.concatenate(term))
+
+
+@pytest.mark.parametrize("N,d,blk", [(1, 64, 16), (1, 128, 64), (3, 128, 128), (17, 64, 16)])
+def test_tiny_sequences_end_to_end(cuda_lib, N, d, blk):
+    # one or a few tokens: a single (partial) block per head, the 128-row
+    # tiles mostly past N; mask -> forward -> backward against the oracle
+    B, H = 2, 2
+    g = torch.Generator().manual_seed(N * 1000 + d + blk)
+    q, k, v, do = (torch.randn(B, H, N, d, generator=g).to(torch.bfloat16) for _ in range(4))
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    rp, ci = cuda_lib.asa_build_mask(qd, kd, blk, cuda_lib.MODE_TOPK, topk=2, keep_diag=1)
+    o, lse = cuda_lib.bsa_forward(qd, kd, vd, blk, rp, ci)
+    dq, dk, dv = cuda_lib.bsa_backward(qd, kd, vd, o, dod, lse, blk, rp, ci)
+    assert cuda_lib.check_device_status() == 0
+    rp_h, ci_h = rp.cpu().numpy().astype(np.int64), ci.cpu().numpy()
+    nb = -(-N // blk)
+    assert rp_h.tolist() == [min(2, nb) * r for r in range(B * H * nb + 1)]
+    qf, kf, vf, dof = W.as_f64(q), W.as_f64(k), W.as_f64(v), W.as_f64(do)
+    o_ref, l_ref = oracle.masked_attention(qf, kf, vf, blk, rp_h, ci_h)
+    from tests._compare import compare_attention
+    compare_attention(o.float().cpu().numpy(), lse.cpu().numpy(), o_ref, l_ref)
+    ref = oracle.attention_backward(qf, kf, vf, dof, blk, rp_h, ci_h)
+    kbar, _ = oracle.masked_attention(qf, kf, kf, blk, rp_h, ci_h)
+    term = d_term(dof, W.as_f64(o.cpu()), kbar, 1.0 / np.sqrt(d))
+    compare_gradients([x.float().cpu().numpy() for x in (dq, dk, dv)], ref, term)
