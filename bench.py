@@ -10,6 +10,7 @@ effective TFLOPS over computed blocks: Σ over kept (q-block, kv-block) pairs of
 4·n_q·n_k·d with valid tokens only, divided by the step time.
 
   python bench.py [--gpus N --steps K --warmup W] [--workload wan|cog|hunyuan|tiny]
+  python bench.py --workload sweep --keep 0.25 --blk 128   # the keep-ratio sweep
   python bench.py --impl reference      # the fp64 CPU oracle on a bounded sample
 
 Under torchrun every rank runs its own replica of the layer (the path has no
@@ -68,7 +69,13 @@ def peaks():
     return dict(FALLBACK), "fallback"
 
 
-def workload(name: str) -> W.Workload:
+def workload(name: str, keep: float = 0.1, blk: int = 64) -> W.Workload:
+    """The named layer; "sweep" is the Wan-shaped layer under top-k with
+    k = floor(keep * nb) at block size blk."""
+    if name == "sweep":
+        if keep not in W.SWEEP_KEEPS or blk not in W.SWEEP_BLKS:
+            raise ValueError(f"sweep points: keep in {W.SWEEP_KEEPS}, blk in {W.SWEEP_BLKS}")
+        return W.sweep(keep, blk)
     return {"wan": W.WAN, "cog": W.COG, "hunyuan": W.HUNYUAN, "tiny": W.TINY}[name]
 
 
@@ -216,7 +223,7 @@ def oracle_step(w: W.Workload, qkv, heads: int):
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    w = workload(args.workload)
+    w = workload(args.workload, args.keep, args.blk)
     if w.source != "asa":
         print(json.dumps({"impl": "reference", "unavailable":
                           "the CPU oracle arm times the ASA workloads only"}), flush=True)
@@ -249,7 +256,7 @@ def run_reference(args, rank, world):
 # ----------------------------------------------------------------------------- GPU
 def run_gpu(args, rank, world, local):
     from block_sparse_attention_asa_b200 import bsa
-    w = workload(args.workload)
+    w = workload(args.workload, args.keep, args.blk)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
@@ -409,7 +416,9 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="bsa", choices=["bsa", "reference"])
-    ap.add_argument("--workload", default="wan", choices=["wan", "cog", "hunyuan", "tiny"])
+    ap.add_argument("--workload", default="wan", choices=["wan", "cog", "hunyuan", "tiny", "sweep"])
+    ap.add_argument("--keep", type=float, default=0.1, help="sweep: keep ratio of the top-k mask")
+    ap.add_argument("--blk", type=int, default=64, help="sweep: block size")
     ap.add_argument("--ref-heads", type=int, default=12,
                     help="heads in the cpu_baseline sample of the GPU arm")
     ap.add_argument("--ref-heads-per-step", type=int, default=1,

@@ -52,3 +52,12 @@ def test_traffic_applies_to_its_kernel_source_only(bench, monkeypatch):
     assert bench.fwd_traffic("no-such-workload") is None
     monkeypatch.setattr(bench, "FWD_TRAFFIC", {("wan2.1_1.3b_asa", "0" * 64): 1})
     assert bench.fwd_traffic("wan2.1_1.3b_asa") is None
+
+
+def test_sweep_workload_selection(bench):
+    w = bench.workload("sweep", 0.25, 128)
+    assert (w.N, w.blk, w.nb, w.topk, w.mode) == (32760, 128, 256, 64, W.MODE_TOPK)
+    assert bench.workload("sweep", 1.0, 64).topk == 512        # the dense end of the sweep
+    assert bench.workload("wan", 0.25, 128) is W.WAN           # keep / blk apply to the sweep only
+    with pytest.raises(ValueError):
+        bench.workload("sweep", 0.3, 64)
