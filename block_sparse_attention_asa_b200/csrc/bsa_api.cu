@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/bsa.h"
@@ -75,13 +76,37 @@ bool make_map(CUtensorMap* m, const void* base, int BH, int N, int d, int rows) 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// ---- per-device one-time settings --------------------------------------------
+// Flags and cached values are atomics: host threads may make their first calls
+// concurrently; repeating the setting is harmless, a data race would not be.
+constexpr int kMaxDevices = 64;
+using DeviceFlags = std::atomic<bool>[kMaxDevices];
+
+// Raise a kernel's dynamic shared-memory limit once per device; `done` is that
+// kernel's flag array.
+template <typename K>
+bool allow_smem(K kernel, int bytes, DeviceFlags& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+  if (dev < kMaxDevices && done[dev].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  if (dev < kMaxDevices) done[dev].store(true, std::memory_order_release);
+  return true;
+}
+
 // ---- forward launch -----------------------------------------------------------
 int sm_count() {
-  static int counts[64] = {};
+  static std::atomic<int> counts[kMaxDevices];
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (counts[dev] == 0) cudaDeviceGetAttribute(&counts[dev], cudaDevAttrMultiProcessorCount, dev);
-  return counts[dev];
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  int n = counts[dev].load(std::memory_order_acquire);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    counts[dev].store(n, std::memory_order_release);
+  }
+  return n;
 }
 
 template <int D, int BLK>
@@ -96,15 +121,8 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   if (!make_map(&mq, q, B * H, N, D, 128) || !make_map(&mk, k, B * H, N, D, BLK) ||
       !make_map(&mv, v, B * H, N, D, BLK))
     return BSA_ERR_CUDA;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(bsa::bsa_fwd_kernel<D, BLK>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-      return BSA_ERR_CUDA;
-    attr_set[dev] = true;
-  }
+  static DeviceFlags smem_set;
+  if (!allow_smem(bsa::bsa_fwd_kernel<D, BLK>, C::SMEM, smem_set)) return BSA_ERR_CUDA;
   bsa::FwdParams p;
   p.B = B;
   p.H = H;
@@ -176,26 +194,13 @@ size_t select_generic_smem(int R, int nb_pad) {
          (size_t)bsa::kSelWarps * 256 * 4 + (size_t)bsa::kSelWarps * 64 * 8;
 }
 
-// Raise a kernel's dynamic shared memory limit once per device.
-template <typename K>
-bool allow_smem(K kernel, int bytes, bool (&done)[64]) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return false;
-  if (dev < 64 && done[dev]) return true;
-  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-      cudaSuccess)
-    return false;
-  if (dev < 64) done[dev] = true;
-  return true;
-}
-
 template <int D, int NCB>
 int launch_select_regs(bsa::SelectParams sp, int BH, cudaStream_t stream) {
   using T = bsa::SelTile<D, NCB>;
   sp.nb_pad = T::NB_PAD;
   sp.rows_per_cta = T::R;
   sp.dk = T::DK;
-  static bool done[64] = {};
+  static DeviceFlags done;
   if (!allow_smem(bsa::asa_select_kernel<D, NCB>, T::SMEM, done)) return BSA_ERR_CUDA;
   dim3 grid(ceil_div(sp.nb, T::R), BH);
   bsa::asa_select_kernel<D, NCB><<<grid, 256, T::SMEM, stream>>>(sp);
@@ -268,7 +273,7 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
       while (R > 1 && select_generic_smem<D>(R, nb_pad) > budget) --R;
       const size_t smem = select_generic_smem<D>(R, nb_pad);
       if (smem > budget) return BSA_ERR_UNSUPPORTED;
-      static bool done[64] = {};
+      static DeviceFlags done;
       if (!allow_smem(bsa::asa_select_generic_kernel<D>, 220 * 1024, done)) return BSA_ERR_CUDA;
       sp.rows_per_cta = R;
       sp.nb_pad = nb_pad;
@@ -288,21 +293,6 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
 }
 
 // ---- backward launches ---------------------------------------------------------
-// Raise a kernel's dynamic shared-memory limit once per device; `done` is the
-// caller's per-kernel flag array.
-template <typename KernelT>
-bool set_smem_once(KernelT kernel, int bytes, bool (&done)[64]) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (!done[dev]) {
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
-        cudaSuccess)
-      return false;
-    done[dev] = true;
-  }
-  return true;
-}
-
 template <int D, int BLK>
 int launch_bwd(const void* q, const void* k, const void* v, const void* dout, int B, int H,
                int N, const int32_t* row_ptr, const int32_t* col_idx, const float* lse,
@@ -320,9 +310,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* dout, in
       !make_map(&qb, q, BH, N, D, BLK) || !make_map(&dob, dout, BH, N, D, BLK) ||
       !make_map(&kb, k, BH, N, D, BLK) || !make_map(&vb, v, BH, N, D, BLK))
     return BSA_ERR_CUDA;
-  static bool dq_set[64] = {}, dkdv_set[64] = {};
-  if (!set_smem_once(bsa::bsa_bwd_dq_kernel<D, BLK>, C::SMEM, dq_set) ||
-      !set_smem_once(bsa::bsa_bwd_dkdv_kernel<D, BLK>, C::SMEM, dkdv_set))
+  static DeviceFlags dq_set, dkdv_set;
+  if (!allow_smem(bsa::bsa_bwd_dq_kernel<D, BLK>, C::SMEM, dq_set) ||
+      !allow_smem(bsa::bsa_bwd_dkdv_kernel<D, BLK>, C::SMEM, dkdv_set))
     return BSA_ERR_CUDA;
   bsa::BwdParams p;
   p.B = B;
