@@ -8,7 +8,7 @@ import torch
 
 import oracle
 from block_sparse_attention_asa_b200 import workloads as W
-from tests._compare import check_csr_valid, compare_masks
+from tests._compare import compare_masks
 
 pytestmark = pytest.mark.gpu
 
