@@ -221,3 +221,19 @@ def test_oracle_masks_pass_the_validator(lib):
     assert bsa.validate_csr(info.row_ptr.astype(np.int32), info.col_idx, w.nb) == -1
     rp, ci = oracle.pattern_mask([0, 1, 2, 3, 4, 5], 1, 6, 300, 16, 2, 64, -1, 1, 1, 1)
     assert bsa.validate_csr(np.asarray(rp, np.int32), np.asarray(ci, np.int32), 19) == -1
+
+
+def test_binding_signatures_match_the_header():
+    # every function the header declares has a ctypes signature in the binding,
+    # with as many arguments as the declaration has parameters
+    import re
+    with open(bsa.HEADER) as f:
+        text = re.sub(r"/\*.*?\*/", "", f.read(), flags=re.S)
+    decls = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(([^;{}]*?)\)\s*;", text)
+    assert decls
+    for name, params in decls:
+        params = " ".join(params.split())
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert name in bsa._SIGNATURES, f"{name} has no binding signature"
+        assert len(bsa._SIGNATURES[name][1]) == n, (name, n, len(bsa._SIGNATURES[name][1]))
+    assert {n for n, _ in decls} == set(bsa._SIGNATURES)
