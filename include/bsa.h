@@ -29,6 +29,16 @@
  *    B*H*nb*nb < 2^31 (the backward also nb <= 4096).  The device must be
  *    sm_100 (B200).
  *
+ * Typical call sequence for one attention layer (device buffers owned by the
+ * caller, all calls on one stream):
+ *   ws  = asa_build_mask_workspace_size(B, H, N, d, blk)     -> allocate ws
+ *   cap = asa_build_mask_max_nnz(B, H, N, blk, mode, ...)    -> col_idx [cap]
+ *   asa_build_mask(q, k, ..., row_ptr, col_idx, cap, ws, ws_bytes, s);
+ *   bsa_forward(q, k, v, ..., row_ptr, col_idx, scale, o, lse, fws, fws_bytes, s);
+ *   (training) bsa_backward(q, k, v, o, dout, lse, ..., dq, dk, dv, bws, bws_bytes, s);
+ *   bsa_check_device_status(s)   -- once per step or when debugging
+ * pattern_mask replaces asa_build_mask for the fixed patterns.
+ *
  * Sources (web pages on the method):
  *  [BLADE]   "BLADE: Block-Sparse Attention Meets Step Distillation for
  *            Efficient Video Generation" (digest: abstract; 技术框架;
