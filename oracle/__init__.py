@@ -42,6 +42,6 @@ check against: its parity beyond that is unpinned.
 """
 from .asa import pool, pooled_probs, select_row, asa_mask, MaskInfo  # noqa: F401
 from .patterns import pattern_row, pattern_mask, keep_token_pair  # noqa: F401
-from .attention import masked_attention, attention_rows  # noqa: F401
+from .attention import masked_attention, attention_rows, attention_probs  # noqa: F401
 from .backward import attention_backward, attention_backward_sampled, mask_transpose  # noqa: F401
 from . import search  # noqa: F401

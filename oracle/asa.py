@@ -66,6 +66,7 @@ class RowSelection:
     mass_at_cut: float    # cumulative p of the kept prefix (before the cap)
     n_selected: int       # blocks kept by the rule (before forcing)
     mass_before_cut: float = 0.0  # cumulative p of the prefix one shorter
+    n_prefix: int = 0     # length of the rule's prefix before the cap
 
 
 def select_row(p_row: np.ndarray, i: int, mode: int, topk: int = 0, mass_tau: float = 0.0,
@@ -93,13 +94,14 @@ def select_row(p_row: np.ndarray, i: int, mode: int, topk: int = 0, mass_tau: fl
         before = prefix(m - 1)
     else:
         raise ValueError(f"unknown mode {mode}")
+    m_prefix = m
     m = min(m, keep_cap(nb, max_keep_ratio))
     chosen = set(int(j) for j in order[:m])
     p_thr = float(p_row[order[m - 1]]) if m > 0 else float("inf")
     if keep_diag:
         chosen.add(int(i))
     chosen.update(range(min(max(n_sink_blocks, 0), nb)))
-    return RowSelection(sorted(chosen), p_thr, mass, m, before)
+    return RowSelection(sorted(chosen), p_thr, mass, m, before, m_prefix)
 
 
 @dataclass
@@ -110,6 +112,7 @@ class MaskInfo:
     mass_at_cut: np.ndarray  # float64 [rows]
     probs: np.ndarray     # float64 [B, H, nb, nb]
     mass_before_cut: np.ndarray = None  # float64 [rows]
+    n_prefix: np.ndarray = None  # int64 [rows]: the rule's prefix length before the cap
 
 
 def asa_mask(q: np.ndarray, k: np.ndarray, blk: int, mode: int, topk: int = 0,
@@ -125,6 +128,7 @@ def asa_mask(q: np.ndarray, k: np.ndarray, blk: int, mode: int, topk: int = 0,
     p_thr = np.empty(rows)
     mass = np.empty(rows)
     before = np.empty(rows)
+    n_prefix = np.empty(rows, dtype=np.int64)
     r = 0
     for b in range(B):
         for h in range(H):
@@ -136,5 +140,6 @@ def asa_mask(q: np.ndarray, k: np.ndarray, blk: int, mode: int, topk: int = 0,
                 p_thr[r] = sel.p_thr
                 mass[r] = sel.mass_at_cut
                 before[r] = sel.mass_before_cut
+                n_prefix[r] = sel.n_prefix
                 r += 1
-    return MaskInfo(row_ptr, np.asarray(cols, dtype=np.int32), p_thr, mass, p, before)
+    return MaskInfo(row_ptr, np.asarray(cols, dtype=np.int32), p_thr, mass, p, before, n_prefix)

@@ -70,3 +70,30 @@ def masked_attention(q, k, v, blk: int, row_ptr, col_idx, scale: float | None = 
         o[b, h, t0:t1] = orow
         lse[b, h, t0:t1] = lrow
     return o, lse
+
+
+def attention_probs(q, k, blk: int, row_ptr, col_idx, scale: float | None = None):
+    """The attention weights P [B, H, N, N] of every query token over every key
+    token: softmax_u(q_t·k_u·scale) over the keys its row lists (u < N), and 0
+    for keys it does not list.  A row that lists nothing is all zeros.
+
+    Dense over N x N: for small sequences only (the per-element rounding bounds
+    of the gradient tests use it).
+    """
+    B, H, n, d = q.shape
+    nb = -(-n // blk)
+    if scale is None or scale <= 0:
+        scale = 1.0 / math.sqrt(d)
+    p = np.zeros((B, H, n, n))
+    for r in range(B * H * nb):
+        i = r % nb
+        bh = r // nb
+        b, h = bh // H, bh % H
+        t0, t1 = i * blk, min(n, (i + 1) * blk)
+        keys = _row_keys(col_idx[row_ptr[r]:row_ptr[r + 1]], blk, n)
+        if keys.size == 0:
+            continue
+        s = (q[b, h, t0:t1] @ k[b, h, keys].T) * scale
+        e = np.exp(s - s.max(axis=1, keepdims=True))
+        p[b, h, t0:t1][:, keys] = e / e.sum(axis=1, keepdims=True)
+    return p

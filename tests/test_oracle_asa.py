@@ -178,3 +178,41 @@ def test_single_token_layer():
     o, lse = oracle.masked_attention(q, k, v, 16, m.row_ptr, m.col_idx)
     np.testing.assert_allclose(o, v, rtol=0, atol=1e-15)
     assert abs(lse[0, 0, 0] - float((q * k).sum()) / 2.0) < 1e-15
+
+
+def test_mask_comparator_exempt_rows():
+    # a mass-mode row whose cut lies at tau is exempt from equality, but must
+    # still be the forced blocks plus a prefix of the (p desc, j asc) order one
+    # block either side of the oracle's: a row with the right count and a wrong
+    # block fails tests/_compare.py
+    from tests._compare import compare_masks, csr_rows
+    rng = np.random.default_rng(8)
+    B, H, N, d, blk = 1, 1, 128, 16, 16
+    nb = N // blk
+    q, k = (rng.standard_normal((B, H, N, d)) for _ in range(2))
+    p = oracle.pooled_probs(q, k, blk)[0, 0, 0]
+    order = np.lexsort((np.arange(nb), -p))
+    tau = math.fsum(p[order[:3]].tolist())       # row 0's cut lands exactly on tau
+    info = oracle.asa_mask(q, k, blk, oracle.asa.MODE_MASS, mass_tau=tau, keep_diag=1)
+    assert info.n_prefix[0] == 3
+    rows = csr_rows(info.row_ptr, info.col_idx)
+    forced = lambda r: [r % nb]
+
+    def check(row0):
+        rs = [sorted(row0)] + rows[1:]
+        rp = np.zeros(len(rs) + 1, dtype=np.int64)
+        rp[1:] = np.cumsum([len(x) for x in rs])
+        ci = np.asarray([c for x in rs for c in x], dtype=np.int32)
+        return compare_masks(rp, ci, info, nb, 1, tau, None, forced)
+
+    for L in (2, 3, 4):
+        got = check(set(int(j) for j in order[:L]) | {0})
+        assert got[3] == (0 if L == 3 else 1)
+    wrong = set(int(j) for j in order[:3]) | {0}
+    wrong = (wrong - {int(order[1])}) | {int(order[-1])}   # same count, wrong block
+    if 0 in (int(order[1]), int(order[-1])):
+        pytest.skip("seed puts the diagonal at the swapped position")
+    with pytest.raises(AssertionError):
+        check(wrong)
+    with pytest.raises(AssertionError):
+        check(set(int(j) for j in order[:6]) | {0})       # two blocks past the cut

@@ -135,3 +135,28 @@ def test_skip_row_is_zero_and_neg_inf():
     assert np.all(o[0, 0, :16] == 0.0) and np.all(np.isneginf(lse[0, 0, :16]))
     assert np.all(o[0, 0, 32:] == 0.0) and np.all(np.isneginf(lse[0, 0, 32:]))
     assert np.all(np.isfinite(lse[0, 0, 16:32]))
+
+
+def test_attention_probs_pins():
+    # P @ V is the oracle's O, kept rows sum to 1 and empty rows to 0; with every
+    # block kept P is torch's softmax of the scaled scores
+    rng = np.random.default_rng(12)
+    B, H, N, d, blk = 1, 2, 37, 16, 8
+    q, k, v = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    nb = -(-N // blk)
+    rows = [[] if r % 3 == 0 else sorted(rng.choice(nb, size=2, replace=False).tolist())
+            for r in range(B * H * nb)]
+    rp = np.zeros(B * H * nb + 1, dtype=np.int64)
+    rp[1:] = np.cumsum([len(c) for c in rows])
+    ci = np.asarray([c for cols in rows for c in cols], dtype=np.int32)
+    p = oracle.attention_probs(q, k, blk, rp, ci)
+    o, lse = oracle.masked_attention(q, k, v, blk, rp, ci)
+    np.testing.assert_allclose(p @ v, o, rtol=0, atol=1e-12)
+    sums = p.sum(axis=-1)
+    np.testing.assert_allclose(sums[np.isfinite(lse)], 1.0, rtol=0, atol=1e-12)
+    assert np.all(sums[~np.isfinite(lse)] == 0)
+    rp_all = np.arange(B * H * nb + 1, dtype=np.int64) * nb
+    ci_all = np.tile(np.arange(nb, dtype=np.int32), B * H * nb)
+    p_all = oracle.attention_probs(q, k, blk, rp_all, ci_all)
+    want = torch.softmax(torch.from_numpy(q) @ torch.from_numpy(k).transpose(-1, -2) / np.sqrt(d), -1)
+    np.testing.assert_allclose(p_all, want.numpy(), rtol=0, atol=1e-12)

@@ -261,3 +261,41 @@ def test_sampled_gradients_equal_the_full_ones():
         np.testing.assert_allclose(dq[r], full[0][b, h, t], rtol=0, atol=1e-12)
         np.testing.assert_allclose(dkv[r][0], full[1][b, h, t], rtol=0, atol=1e-12)
         np.testing.assert_allclose(dkv[r][1], full[2][b, h, t], rtol=0, atol=1e-12)
+
+
+def _bf16(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16).double().numpy()
+
+
+def test_zero_gradient_bound_single_key():
+    # one token per head: the exact dQ and dK are zero.  A kernel forming dP and
+    # D as fp32 sums in different orders (sequential vs reversed) and D from an
+    # Ô that is one bf16 ulp off in one element stays within the rounding bound
+    # of tests/_compare.py; a dropped D term or a planted 1e-3 does not.
+    from tests._compare import compare_gradients, zero_gradient_bounds
+    B, H, N, d, blk = 2, 2, 1, 64, 16
+    q, k, v, do = (_bf16(x) for x in _qkv(B, H, N, d, 31))
+    rp, ci = _full_csr(B, H, 1)
+    scale = 1 / math.sqrt(d)
+    ref = oracle.attention_backward(q, k, v, do, blk, rp, ci)
+    assert np.all(ref[0] == 0) and np.all(ref[1] == 0)
+    o_ref, _ = oracle.masked_attention(q, k, v, blk, rp, ci)
+    o_hat = o_ref.copy()
+    o_hat[0, 0, 0, 3] = _bf16(o_hat[0, 0, 0, 3] * (1 + 2.0 ** -7))[()]
+    prod_v = (do * v).astype(np.float32)
+    prod_o = (do * o_hat).astype(np.float32)
+    dp32 = np.cumsum(prod_v, axis=-1, dtype=np.float32)[..., -1]
+    d32 = np.cumsum(prod_o[..., ::-1], axis=-1, dtype=np.float32)[..., -1]
+    ds = _bf16(dp32 - d32)[..., None]
+    got = (_bf16(scale * ds * k), _bf16(scale * ds * q), _bf16(ref[2]))
+    probs = oracle.attention_probs(q, k, blk, rp, ci)
+    zb = zero_gradient_bounds(q, k, v, do, o_hat, o_ref, probs, scale)
+    assert np.max(np.abs(got[0])) > 0     # the emulated rounding is not zero
+    compare_gradients(got, ref, None, zb)
+    with pytest.raises(AssertionError):   # without the bound: exact zero demanded
+        compare_gradients(got, ref, None, None)
+    dropped_d = _bf16(scale * dp32[..., None] * k)
+    for g in ((dropped_d, got[1], got[2]), (got[0] + 1e-3, got[1], got[2]),
+              (got[0], got[1] - 1e-3, got[2])):
+        with pytest.raises(AssertionError):
+            compare_gradients(g, ref, None, zb)
