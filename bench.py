@@ -13,6 +13,13 @@ effective TFLOPS over computed blocks: Σ over kept (q-block, kv-block) pairs of
   python bench.py --workload sweep --keep 0.25 --blk 128   # the keep-ratio sweep
   python bench.py --impl reference      # the fp64 CPU oracle on a bounded sample
 
+On one GPU the same line also carries, under "extra", the other layers timed
+the same way with fewer steps (the CogVideoX-shaped layer, the HunyuanVideo-
+shaped layer with its fixed patterns, the Wan-shaped layer under the 3D tile,
+and the ten keep-ratio x block-size sweep
+points on the Wan shape, mask time apart from forward time) and the backward on
+the headline layer (--no-extra skips them).
+
 Under torchrun every rank runs its own replica of the layer (the path has no
 cross-GPU exchange); the timed region is bracketed by barriers and the maximum
 over ranks is reported.
@@ -43,9 +50,9 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 
 # DRAM bytes (read + write) per bsa_fwd_kernel launch, from one ncu capture of
-# the bench's own command (profiles/bsa_fwd_kernel_wan.md), keyed by workload and
-# by the sha256 of the kernel source the capture ran: once the kernel changes,
-# the figure no longer applies and the bench reports null.
+# the bench's own command, keyed by workload and by the sha256 of the kernel
+# source the capture ran: once the kernel changes, the figure no longer applies
+# and the bench reports null.
 FWD_TRAFFIC = {
     ("wan2.1_1.3b_asa", "96289554c31f2322f6a5e5b32e686dc6dd3aafabd8be7fdf376cfb7edc0f9c88"):
         309146368 + 85984768,
@@ -76,7 +83,8 @@ def workload(name: str, keep: float = 0.1, blk: int = 64) -> W.Workload:
         if keep not in W.SWEEP_KEEPS or blk not in W.SWEEP_BLKS:
             raise ValueError(f"sweep points: keep in {W.SWEEP_KEEPS}, blk in {W.SWEEP_BLKS}")
         return W.sweep(keep, blk)
-    return {"wan": W.WAN, "cog": W.COG, "hunyuan": W.HUNYUAN, "tiny": W.TINY}[name]
+    return {"wan": W.WAN, "cog": W.COG, "hunyuan": W.HUNYUAN, "tiny": W.TINY,
+            "tile3d": W.WAN_TILE3D}[name]
 
 
 def block_flops(w: W.Workload, row_ptr: np.ndarray, col_idx: np.ndarray) -> float:
@@ -254,91 +262,179 @@ def run_reference(args, rank, world):
 
 
 # ----------------------------------------------------------------------------- GPU
+class Layer:
+    """Device buffers of one workload and the two launches of its step (the mask,
+    then bsa_forward), through the C ABI."""
+
+    def __init__(self, bsa, w: W.Workload, dev, qkv=None):
+        self.bsa, self.w, self.dev = bsa, w, dev
+        if qkv is None:
+            self.host = W.make_qkv(w)
+            qkv = tuple(t.to(dev) for t in self.host)
+        else:
+            self.host = None
+        self.q, self.k, self.v = qkv
+        B, H, N, d = self.q.shape
+        self.rows = B * H * w.nb
+        if w.source == "asa":
+            cap = bsa.asa_max_nnz(B, H, N, w.blk, w.mode, w.topk, w.max_keep_ratio, w.keep_diag,
+                                  w.n_sink_blocks)
+            self.ws = torch.empty(bsa.asa_workspace_size(B, H, N, d, w.blk), dtype=torch.uint8,
+                                  device=dev)
+            self.hp = None
+        else:
+            _, ci_probe = bsa.pattern_mask(w.head_pattern, B, H, N, w.blk, w.band_w,
+                                           w.frame_tokens, w.f_lo, w.f_hi, w.stripe_blocks,
+                                           w.tile_global_frames, device=dev)
+            cap = int(ci_probe.numel())
+            del ci_probe
+            self.ws = None
+            import ctypes
+            self.hp = (ctypes.c_int32 * H)(*w.head_pattern)
+        self.row_ptr = torch.empty(self.rows + 1, dtype=torch.int32, device=dev)
+        self.col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
+        self.fws = torch.empty(max(bsa.forward_workspace_size(B, H, N, d, w.blk), 4),
+                               dtype=torch.uint8, device=dev)
+        self.o = torch.empty_like(self.q)
+        self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        # kernels per step: pool, select, scan, expand (ASA) or pattern + scan
+        self.launches = (4 if w.source == "asa" else 3) + 1
+
+    def mask(self):
+        w, b = self.w, self.bsa
+        B, H, N, _ = self.q.shape
+        if w.source == "asa":
+            b.asa_build_mask_into(self.q, self.k, w.blk, w.mode, w.topk, w.mass_tau,
+                                  w.max_keep_ratio, w.keep_diag, w.n_sink_blocks, 0.0,
+                                  self.row_ptr, self.col_idx, self.ws)
+        else:
+            b.pattern_mask_into(self.hp, B, H, N, w.blk, w.band_w, w.frame_tokens, w.f_lo,
+                                w.f_hi, w.stripe_blocks, w.tile_global_frames, self.row_ptr,
+                                self.col_idx)
+
+    def forward(self):
+        self.bsa.bsa_forward_into(self.q, self.k, self.v, self.w.blk, self.row_ptr, self.col_idx,
+                                  self.o, self.lse, workspace=self.fws)
+
+    def mask_bytes(self, nnz: int) -> float:
+        csr = 4.0 * (self.rows + 1) + 4.0 * nnz
+        return csr + (2.0 * self.q.numel() * 2 if self.w.source == "asa" else 0.0)
+
+
+def check_status(bsa, where: str):
+    st = bsa.check_device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {where}: {bsa.status_string(st)}")
+
+
+def time_layer(layer: Layer, steps: int, warmup: int, local: int, world: int, stream):
+    """Warm-up, then `steps` back-to-back steps with per-kernel CUDA events on the
+    launching stream and the SM clock sampled inside the timed region."""
+    bsa, w = layer.bsa, layer.w
+    for _ in range(warmup):
+        layer.mask()
+        layer.forward()
+    check_status(bsa, "after warm-up")
+    rp_h = layer.row_ptr.cpu().numpy()
+    ci_h = layer.col_idx[:int(rp_h[-1])].cpu().numpy()
+    flops = block_flops(w, rp_h, ci_h)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        clk.mark_start()
+        t0.record(stream)
+        for s in range(steps):
+            ev[s][0].record(stream)
+            layer.mask()
+            ev[s][1].record(stream)
+            layer.forward()
+            ev[s][2].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        clk.mark_end()
+    barrier(world)
+    check_status(bsa, "after timing")
+    return {
+        "total_ms": t0.elapsed_time(t1),
+        "mask_ms": [e[0].elapsed_time(e[1]) for e in ev],
+        "fwd_ms": [e[1].elapsed_time(e[2]) for e in ev],
+        "clocks": clk.summary(), "flops": flops, "nnz": int(rp_h[-1]),
+        "keep": float(rp_h[-1]) / (layer.rows * w.nb),
+    }
+
+
+def layer_summary(layer: Layer, t: dict, pk: dict, steps: int) -> dict:
+    """Per-layer figures of one timing: ms, TFLOPS and the fractions of the peaks."""
+    fwd = statistics.mean(t["fwd_ms"])
+    mask = statistics.mean(t["mask_ms"])
+    tf = t["flops"] / (fwd * 1e-3) / 1e12
+    gbs = layer.mask_bytes(t["nnz"]) / (mask * 1e-3) / 1e9
+    return {
+        "ms_per_layer": t["total_ms"] / steps, "ms_mask": mask, "ms_forward": fwd,
+        "forward_tflops": tf, "frac": tf / float(pk["bf16_tflops"]),
+        "mask_kernel": "asa_build_mask" if layer.w.source == "asa" else "pattern_mask",
+        "mask_gbs": gbs, "mask_frac": gbs / float(pk["hbm_gbs"]),
+        "keep_ratio": t["keep"], "block_flops": t["flops"], "steps": steps,
+        "clocks": t["clocks"],
+    }
+
+
+def time_backward(bsa, layer: Layer, flops: float, pk: dict, iters: int = 10, warmup: int = 3):
+    """bsa_backward on the layer's mask, O and LSE for a seeded dO (CUDA events,
+    median of `iters` calls).  Flops at the usual 2.5x the forward's block flops."""
+    q, k, v, w = layer.q, layer.k, layer.v, layer.w
+    B, H, N, d = q.shape
+    g = torch.Generator(device=q.device).manual_seed(5)
+    dout = torch.randn(q.shape, generator=g, device=q.device).to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(max(bsa.backward_workspace_size(B, H, N, d, w.blk), 4), dtype=torch.uint8,
+                     device=q.device)
+
+    def call():
+        bsa.bsa_backward_into(q, k, v, layer.o, dout, layer.lse, w.blk, layer.row_ptr,
+                              layer.col_idx, dq, dk, dv, 0.0, ws)
+    for _ in range(warmup):
+        call()
+    check_status(bsa, "after backward warm-up")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(iters)]
+    torch.cuda.synchronize()
+    for a, b in evs:
+        a.record()
+        call()
+        b.record()
+    torch.cuda.synchronize()
+    check_status(bsa, "after backward timing")
+    ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+    tf = 2.5 * flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "ms_backward": ms, "tflops_2p5x": tf,
+            "frac": tf / float(pk["bf16_tflops"]), "flop_convention": "2.5x forward block flops",
+            "iters": iters}
+
+
 def run_gpu(args, rank, world, local):
     from block_sparse_attention_asa_b200 import bsa
     w = workload(args.workload, args.keep, args.blk)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    q_h, k_h, v_h = W.make_qkv(w)
-    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    layer = Layer(bsa, w, dev)
+    q_h, k_h, v_h = layer.host
+    q, o, lse = layer.q, layer.o, layer.lse
     B, H, N, d = q.shape
-    nb = w.nb
-    rows = B * H * nb
-    if w.source == "asa":
-        cap = bsa.asa_max_nnz(B, H, N, w.blk, w.mode, w.topk, w.max_keep_ratio, w.keep_diag,
-                              w.n_sink_blocks)
-        ws = torch.empty(bsa.asa_workspace_size(B, H, N, d, w.blk), dtype=torch.uint8, device=dev)
-    else:
-        _, ci_probe = bsa.pattern_mask(w.head_pattern, B, H, N, w.blk, w.band_w, w.frame_tokens,
-                                       w.f_lo, w.f_hi, w.stripe_blocks, w.tile_global_frames,
-                                       device=dev)
-        cap = int(ci_probe.numel())
-        ws = None
-    row_ptr = torch.empty(rows + 1, dtype=torch.int32, device=dev)
-    col_idx = torch.empty(max(cap, 1), dtype=torch.int32, device=dev)
-    fws = torch.empty(max(bsa.forward_workspace_size(B, H, N, d, w.blk), 4), dtype=torch.uint8,
-                      device=dev)
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    hp = None
-    if w.source == "pattern":
-        import ctypes
-        hp = (ctypes.c_int32 * H)(*w.head_pattern)
-
-    def mask():
-        if w.source == "asa":
-            bsa.asa_build_mask_into(q, k, w.blk, w.mode, w.topk, w.mass_tau, w.max_keep_ratio,
-                                    w.keep_diag, w.n_sink_blocks, 0.0, row_ptr, col_idx, ws)
-        else:
-            bsa.pattern_mask_into(hp, B, H, N, w.blk, w.band_w, w.frame_tokens, w.f_lo, w.f_hi,
-                                  w.stripe_blocks, w.tile_global_frames, row_ptr, col_idx)
-
-    def forward():
-        bsa.bsa_forward_into(q, k, v, w.blk, row_ptr, col_idx, o, lse, workspace=fws)
-
-    launches_per_step = (4 if w.source == "asa" else 3) + 1
-    for _ in range(args.warmup):
-        mask()
-        forward()
-    st = bsa.check_device_status()
-    if st != 0:
-        raise RuntimeError(f"device status after warm-up: {bsa.status_string(st)}")
-    rp_h = row_ptr.cpu().numpy()
-    ci_h = col_idx[:int(rp_h[-1])].cpu().numpy()
-    flops = block_flops(w, rp_h, ci_h)
-    keep = float(rp_h[-1]) / (rows * nb)
+    rows = layer.rows
 
     # ---- timed region: K steps, per-kernel events on the launching stream
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t_all0 = torch.cuda.Event(enable_timing=True)
-        t_all1 = torch.cuda.Event(enable_timing=True)
-        clk.mark_start()
-        t_all0.record(stream)
-        for s in range(args.steps):
-            ev[s][0].record(stream)
-            mask()
-            ev[s][1].record(stream)
-            forward()
-            ev[s][2].record(stream)
-        t_all1.record(stream)
-        torch.cuda.synchronize()
-        clk.mark_end()
-    barrier(world)
-    total_ms = t_all0.elapsed_time(t_all1)
-    mask_ms = [e[0].elapsed_time(e[1]) for e in ev]
-    fwd_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = barrier_max(total_ms, world)
+    t = time_layer(layer, args.steps, args.warmup, local, world, stream)
+    total_ms = barrier_max(t["total_ms"], world)
     ms_step = total_ms / args.steps
-    st = bsa.check_device_status()
-    if st != 0:
-        raise RuntimeError(f"device status after timing: {bsa.status_string(st)}")
+    flops, keep, nnz = t["flops"], t["keep"], t["nnz"]
 
     # ---- end to end through the public API with host buffers (pinned), copies timed
-    q_p, k_p, v_p = (t.pin_memory() for t in (q_h, k_h, v_h))
+    q_p, k_p, v_p = (x.pin_memory() for x in (q_h, k_h, v_h))
     o_p = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     lse_p = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     e2e_steps = max(1, min(args.steps, 20))
@@ -348,11 +444,11 @@ def run_gpu(args, rank, world, local):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        q.copy_(q_p, non_blocking=True)
-        k.copy_(k_p, non_blocking=True)
-        v.copy_(v_p, non_blocking=True)
-        mask()
-        forward()
+        layer.q.copy_(q_p, non_blocking=True)
+        layer.k.copy_(k_p, non_blocking=True)
+        layer.v.copy_(v_p, non_blocking=True)
+        layer.mask()
+        layer.forward()
         o_p.copy_(o, non_blocking=True)
         lse_p.copy_(lse, non_blocking=True)
     e1.record(stream)
@@ -362,13 +458,9 @@ def run_gpu(args, rank, world, local):
     d2h = o.numel() * o.element_size() + lse.numel() * lse.element_size()
 
     pk, pk_kind = peaks()
-    fwd_avg = statistics.mean(fwd_ms)
-    mask_avg = statistics.mean(mask_ms)
-    achieved = flops / (fwd_avg * 1e-3) / 1e12
+    summ = layer_summary(layer, t, pk, args.steps)
+    achieved = summ["forward_tflops"]
     peak = float(pk["bf16_tflops"])
-    mask_bytes = (2.0 * q.numel() * 2 + 4.0 * (rows + 1) + 4.0 * rp_h[-1]) if w.source == "asa" \
-        else (4.0 * (rows + 1) + 4.0 * rp_h[-1])
-    mask_gbs = mask_bytes / (mask_avg * 1e-3) / 1e9
     value = flops * world / (ms_step * 1e-3) / 1e12
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
@@ -384,21 +476,24 @@ def run_gpu(args, rank, world, local):
             "l2": f"inputs larger than L2: Q+K+V = {3 * q.numel() * 2 / 1e6:.0f} MB per step",
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
         },
-        "ms_mask": mask_avg, "ms_forward": fwd_avg,
+        "ms_mask": summ["ms_mask"], "ms_forward": summ["ms_forward"],
         "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel", "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_kind": f"{pk_kind} bf16 burst", "traffic": fwd_traffic(w.name),
                      "traffic_unit": "bytes per launch (ncu dram read + write)",
                      "frac_of_sustained": achieved / float(pk.get("bf16_tflops_sustained", peak)),
                      "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS},
-        "mask_roofline": {"bound": "hbm", "achieved": mask_gbs, "peak": float(pk["hbm_gbs"]),
-                          "unit": "GB/s", "frac": mask_gbs / float(pk["hbm_gbs"]),
-                          "frac_of_8tbs": mask_gbs / DATASHEET_HBM_GBS},
+        "mask_roofline": {"bound": "hbm", "kernel": summ["mask_kernel"],
+                          "achieved": summ["mask_gbs"], "peak": float(pk["hbm_gbs"]),
+                          "unit": "GB/s", "frac": summ["mask_frac"],
+                          "frac_of_8tbs": summ["mask_gbs"] / DATASHEET_HBM_GBS},
         "e2e": {"value": flops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "clocks": clk.summary(),
-        "gpu_launches": launches_per_step * args.steps,
+        "clocks": t["clocks"],
+        "gpu_launches": layer.launches * args.steps,
     }
+    if world == 1 and not args.no_extra:
+        out["extra"] = run_extra(bsa, args, layer, flops, pk, local, stream)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and w.source == "asa":
         heads = max(1, min(w.H, args.ref_heads))
         dt, fl = oracle_step(w, oracle_inputs(w, heads), heads)
@@ -410,13 +505,49 @@ def run_gpu(args, rank, world, local):
         print(json.dumps(out), flush=True)
 
 
+def run_extra(bsa, args, head_layer: Layer, head_flops: float, pk: dict, local: int, stream):
+    """The other layers the workloads name, each timed like the headline (fewer
+    steps), plus the backward on the headline layer.  Keys: the workload names,
+    "sweep" (keep ratio x block size on the Wan shape, inputs shared with the
+    headline layer when it is that shape) and "backward"."""
+    ex = {}
+    dev = head_layer.dev
+    steps, warm = args.extra_steps, 3
+    try:
+        ex["backward"] = time_backward(bsa, head_layer, head_flops, pk)
+    except RuntimeError as e:
+        ex["backward"] = {"error": str(e)}
+    wan_qkv = (head_layer.q, head_layer.k, head_layer.v) if head_layer.w.name == W.WAN.name else None
+    for wl in (W.COG, W.HUNYUAN, W.WAN_TILE3D):
+        if wl.name == head_layer.w.name:
+            continue
+        same = wan_qkv is not None and (wl.B, wl.H, wl.N, wl.d, wl.seed, wl.scale, wl.pe) == (
+            W.WAN.B, W.WAN.H, W.WAN.N, W.WAN.d, W.WAN.seed, W.WAN.scale, W.WAN.pe)
+        lay = Layer(bsa, wl, dev, wan_qkv if same else None)
+        ex[wl.name] = layer_summary(lay, time_layer(lay, steps, warm, local, 1, stream), pk, steps)
+        del lay
+        torch.cuda.empty_cache()
+    sw = {}
+    for blk in W.SWEEP_BLKS:
+        for kp in W.SWEEP_KEEPS:
+            ws = W.sweep(kp, blk)
+            lay = Layer(bsa, ws, dev, wan_qkv)
+            if wan_qkv is None:
+                wan_qkv = (lay.q, lay.k, lay.v)
+            sw[f"keep{kp}_blk{blk}"] = layer_summary(lay, time_layer(lay, steps, warm, local, 1,
+                                                                     stream), pk, steps)
+            del lay
+    ex["sweep"] = sw
+    return ex
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="bsa", choices=["bsa", "reference"])
-    ap.add_argument("--workload", default="wan", choices=["wan", "cog", "hunyuan", "tiny", "sweep"])
+    ap.add_argument("--workload", default="wan", choices=["wan", "cog", "hunyuan", "tiny", "tile3d", "sweep"])
     ap.add_argument("--keep", type=float, default=0.1, help="sweep: keep ratio of the top-k mask")
     ap.add_argument("--blk", type=int, default=64, help="sweep: block size")
     ap.add_argument("--ref-heads", type=int, default=12,
@@ -424,6 +555,9 @@ def main():
     ap.add_argument("--ref-heads-per-step", type=int, default=1,
                     help="heads per step of the --impl reference arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other layers, the sweep and the backward (1 GPU only)")
+    ap.add_argument("--extra-steps", type=int, default=5, help="timed steps of each extra layer")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

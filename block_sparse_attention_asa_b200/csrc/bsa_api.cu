@@ -501,10 +501,12 @@ int64_t asa_build_mask_max_nnz(int B, int H, int N, int blk, int mode, int topk,
   return (int64_t)B * H * nb * per;
 }
 
-int asa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int blk, int mode,
-                   int topk, float mass_tau, float max_keep_ratio, int keep_diag,
-                   int n_sink_blocks, float softmax_scale, int32_t* row_ptr, int32_t* col_idx,
-                   int64_t col_capacity, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+// The argument checks shared by asa_build_mask and asa_build_mask_noalloc
+// (everything but the workspace).
+static int asa_mask_arg_checks(const void* q, const void* k, int B, int H, int N, int d, int blk,
+                               int mode, int topk, float mass_tau, float max_keep_ratio,
+                               int n_sink_blocks, float softmax_scale, const int32_t* row_ptr,
+                               const int32_t* col_idx, int64_t col_capacity) {
   if (!q || !k || !row_ptr || (!col_idx && col_capacity > 0) || col_capacity < 0)
     return BSA_ERR_INVALID_ARG;
   int rc = common_shape_checks(B, H, N, blk);
@@ -516,8 +518,17 @@ int asa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int
   if (mode == BSA_MODE_MASS && !(mass_tau > 0.f && mass_tau <= 1.f)) return BSA_ERR_INVALID_ARG;
   if (!(max_keep_ratio <= 1.0f) || std::isnan(softmax_scale)) return BSA_ERR_INVALID_ARG;
   if (n_sink_blocks < 0) return BSA_ERR_INVALID_ARG;
-  const long long nb = (N + blk - 1) / blk;
-  if (nb > 65536) return BSA_ERR_UNSUPPORTED;
+  if ((N + blk - 1) / blk > 65536) return BSA_ERR_UNSUPPORTED;
+  return BSA_OK;
+}
+
+int asa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int blk, int mode,
+                   int topk, float mass_tau, float max_keep_ratio, int keep_diag,
+                   int n_sink_blocks, float softmax_scale, int32_t* row_ptr, int32_t* col_idx,
+                   int64_t col_capacity, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  const int rc = asa_mask_arg_checks(q, k, B, H, N, d, blk, mode, topk, mass_tau, max_keep_ratio,
+                                     n_sink_blocks, softmax_scale, row_ptr, col_idx, col_capacity);
+  if (rc != BSA_OK) return rc;
   const AsaLayout L = asa_layout(B, H, N, d, blk);
   if (!workspace || ws_bytes < L.total || !aligned(workspace, 256)) return BSA_ERR_WORKSPACE;
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
@@ -731,19 +742,10 @@ extern "C" int asa_build_mask_noalloc(const void* q, const void* k, int B, int H
                                       float max_keep_ratio, int keep_diag, int n_sink_blocks,
                                       float softmax_scale, int32_t* row_ptr, int32_t* col_idx,
                                       int64_t col_capacity, bsa_stream_t stream) {
-  // same argument checks as asa_build_mask, minus the caller's workspace
-  if (!q || !k || !row_ptr || (!col_idx && col_capacity > 0) || col_capacity < 0)
-    return BSA_ERR_INVALID_ARG;
-  int rc = common_shape_checks(B, H, N, blk);
+  // the same argument checks as asa_build_mask, minus the caller's workspace
+  const int rc = asa_mask_arg_checks(q, k, B, H, N, d, blk, mode, topk, mass_tau, max_keep_ratio,
+                                     n_sink_blocks, softmax_scale, row_ptr, col_idx, col_capacity);
   if (rc != BSA_OK) return rc;
-  if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
-  if (!aligned(q, 16) || !aligned(k, 16)) return BSA_ERR_UNSUPPORTED;
-  if (mode != BSA_MODE_TOPK && mode != BSA_MODE_MASS) return BSA_ERR_INVALID_ARG;
-  if (mode == BSA_MODE_TOPK && topk < 1) return BSA_ERR_INVALID_ARG;
-  if (mode == BSA_MODE_MASS && !(mass_tau > 0.f && mass_tau <= 1.f)) return BSA_ERR_INVALID_ARG;
-  if (!(max_keep_ratio <= 1.0f) || std::isnan(softmax_scale)) return BSA_ERR_INVALID_ARG;
-  if (n_sink_blocks < 0) return BSA_ERR_INVALID_ARG;
-  if ((N + blk - 1) / blk > 65536) return BSA_ERR_UNSUPPORTED;
   // the scratch this shape needs must fit the fixed array
   if (asa_layout(B, H, N, d, blk).total > static_cast<size_t>(BSA_ASA_NOALLOC_MAX_WORKSPACE))
     return BSA_ERR_WORKSPACE;

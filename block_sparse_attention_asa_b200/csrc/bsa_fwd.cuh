@@ -12,8 +12,10 @@
 // step with some masked work beats exact 64-row tiles.
 //
 // Persistent CTAs (one per SM), each running TWO independent item slots (A, B)
-// so that one slot's softmax overlaps the other slot's MMAs.  Items are dealt
-// round-robin: slot X of CTA c takes items 2c+X, 2c+X+2G, ... (G = grid size).
+// so that one slot's softmax overlaps the other slot's MMAs.  Slot X of CTA c
+// starts on item 2c+X; every later item comes from a grid-wide counter, so the
+// SMs that run faster take more items (without a counter, items 2c+X+2kG of a
+// static deal, G = grid size).
 //
 // Warp roles (640 threads, 20 warps):
 //   warp 3      scheduler: per item builds the q-block bitmaps of its CSR rows

@@ -188,6 +188,14 @@ HUNYUAN = Workload(name="hunyuanvideo_patterns", B=1, H=24, d=128, frames=33, he
                    stripe_blocks=4)
 
 
+# The Efficient-vDiT 3D attention tile ("3.1 注意力图块化") on the Wan shape:
+# every head keeps the blocks that share a frame with the query block, plus the
+# blocks of the first frame (one global frame), in the given token order.
+WAN_TILE3D = Workload(name="wan2.1_1.3b_tile3d", B=1, H=12, d=128, frames=21, height=30,
+                      width=52, blk=64, seed=1, scale=0.5, source="pattern",
+                      head_pattern=tuple([PATTERN_TILE3D] * 12), tile_global_frames=1)
+
+
 def sweep(keep: float, blk: int) -> Workload:
     """Wan-shaped layer, top-k with k = floor(keep * nb)."""
     nb = -(-(21 * 30 * 52) // blk)
@@ -198,4 +206,4 @@ def sweep(keep: float, blk: int) -> Workload:
 
 SWEEP_KEEPS = (1.0, 0.5, 0.25, 0.1, 0.05)
 SWEEP_BLKS = (64, 128)
-ALL = {w.name: w for w in (TINY, WAN, COG, HUNYUAN)}
+ALL = {w.name: w for w in (TINY, WAN, COG, HUNYUAN, WAN_TILE3D)}

@@ -144,6 +144,17 @@ def test_forward_hunyuan_patterns_sampled(cuda_lib):
     _run_and_compare(cuda_lib, q, k, v, w.blk, rp.cpu().numpy(), ci.cpu().numpy(), rows=rows)
 
 
+def test_forward_wan_tile3d_sampled(cuda_lib):
+    # the 3D-tile layer: every head keeps its own frames' blocks and frame 0's
+    w = W.WAN_TILE3D
+    q, k, v = W.make_qkv(w)
+    rp, ci = cuda_lib.pattern_mask(w.head_pattern, w.B, w.H, w.N, w.blk, w.band_w, w.frame_tokens,
+                                   w.f_lo, w.f_hi, w.stripe_blocks, w.tile_global_frames)
+    rng = np.random.default_rng(13)
+    rows = sorted(set(rng.choice(w.H * w.nb, size=96, replace=False).tolist() + [0, w.nb - 1]))
+    _run_and_compare(cuda_lib, q, k, v, w.blk, rp.cpu().numpy(), ci.cpu().numpy(), rows=rows)
+
+
 @pytest.mark.parametrize("keep", [1.0, 0.1])
 @pytest.mark.parametrize("blk", W.SWEEP_BLKS)
 def test_forward_sweep_sampled(cuda_lib, keep, blk):

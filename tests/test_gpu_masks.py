@@ -46,6 +46,33 @@ def test_pattern_mask_hunyuan_bit_exact(cuda_lib):
     assert np.array_equal(ci.cpu().numpy(), oci)
 
 
+def test_pattern_mask_tile3d_hand_example(cuda_lib):
+    # the hand-derived 3D-tile rows of tests/golden/tile3d_example.json (frames
+    # that straddle blocks), for 0, 1 and 2 global frames
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "tile3d_example.json")) as f:
+        g = json.load(f)
+    n, S, blk = g["N"], g["frame_tokens"], g["blk"]
+    nb = -(-n // blk)
+    for gf, rows in g["rows"].items():
+        rp, ci = cuda_lib.pattern_mask([W.PATTERN_TILE3D], 1, 1, n, blk, 0, S, 0, 0, 0, int(gf))
+        assert cuda_lib.check_device_status() == 0
+        rp, ci = rp.cpu().numpy(), ci.cpu().numpy()
+        assert [ci[rp[i]:rp[i + 1]].tolist() for i in range(nb)] == rows
+
+
+def test_pattern_mask_wan_tile3d_bit_exact(cuda_lib):
+    w = W.WAN_TILE3D
+    rp, ci = cuda_lib.pattern_mask(w.head_pattern, w.B, w.H, w.N, w.blk, w.band_w, w.frame_tokens,
+                                   w.f_lo, w.f_hi, w.stripe_blocks, w.tile_global_frames)
+    assert cuda_lib.check_device_status() == 0
+    orp, oci = oracle.pattern_mask(w.head_pattern, w.B, w.H, w.N, w.blk, w.band_w, w.frame_tokens,
+                                   w.f_lo, w.f_hi, w.stripe_blocks, w.tile_global_frames)
+    assert np.array_equal(rp.cpu().numpy().astype(np.int64), orp)
+    assert np.array_equal(ci.cpu().numpy(), oci)
+
+
 def test_pattern_mask_capacity_reported(cuda_lib):
     import ctypes
     lib = cuda_lib.load()

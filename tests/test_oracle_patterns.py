@@ -74,3 +74,20 @@ def test_pattern_mask_replicates_over_batch_and_skip_rows_empty():
         assert row(1 * nb + i) == []
         assert row(0 * nb + i) == list(range(nb))
     assert rp[0] == 0 and np.all(np.diff(rp) >= 0)
+
+
+def test_tile3d_hand_example_not_frame_aligned():
+    # tests/golden/tile3d_example.json: rows derived by hand from the token-level
+    # reading, for frames (6 tokens) that straddle the blocks (4 tokens) and a
+    # partial last frame and block
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "tile3d_example.json")) as f:
+        g = json.load(f)
+    n, S, blk = g["N"], g["frame_tokens"], g["blk"]
+    nb = -(-n // blk)
+    for gf, rows in g["rows"].items():
+        got = [oracle.pattern_row(TILE3D, i, nb, n, blk, 0, S, 0, 0, 0, int(gf)) for i in range(nb)]
+        assert got == rows, (gf, got)
+        rp, ci = oracle.pattern_mask([TILE3D], 1, 1, n, blk, 0, S, 0, 0, 0, int(gf))
+        assert [ci[rp[i]:rp[i + 1]].tolist() for i in range(nb)] == rows
