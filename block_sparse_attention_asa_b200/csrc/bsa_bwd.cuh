@@ -29,10 +29,11 @@
 // No atomics: each gradient row is written once by the item that owns it, so
 // the result does not depend on scheduling.
 //
-// Warp roles (256 threads, one item per CTA): all eight warps first build the
-// item's block list; then warp 0 is the producer (TMA), warp 1 the MMA issuer
-// and TMEM owner, warps 4-7 the element-wise step and the epilogue (warp w
-// owns TMEM lane quarter w % 4; one tile row per thread).
+// Warp roles (kBwdThreads threads, one item per CTA): all warps first build
+// the item's block list; then warp 0 is the producer (TMA), warp 1 the MMA
+// issuer and TMEM owner, warps 4.. the element-wise step and the epilogue
+// (warp w owns TMEM lane quarter w % 4 and one contiguous part of the 128
+// columns; one tile row per thread).
 //
 // TMEM columns: S [0,128), dP [128,256), first accumulator [256,256+D),
 // second accumulator [384,384+D).
@@ -50,7 +51,20 @@
 
 namespace bsa {
 
-constexpr int kBwdThreads = 256;
+// Element-wise warps: kBwdEltWarps / 4 per TMEM lane quarter, each taking a
+// contiguous part of the 128 columns of its rows.
+constexpr int kBwdEltWarps = 8;
+constexpr int kBwdParts = kBwdEltWarps / 4;
+constexpr int kBwdCols = 128 / kBwdParts;          // columns per element-wise warp
+constexpr int kBwdThreads = (4 + kBwdEltWarps) * 32;
+static_assert(kBwdCols % 32 == 0, "a warp's columns come in 32-column loads");
+
+// TMEM column of the bf16 pair holding column c (0..127) of a 128-wide S or dP
+// after the element-wise pass: each warp part packs its columns into the first
+// half of its own column range, so no part writes columns another part reads.
+__host__ __device__ constexpr int packed_col(int c) {
+  return (c / kBwdCols) * kBwdCols + (c % kBwdCols) / 2;
+}
 constexpr int kBwdMaxNb = 4096;    // blocks per head (the item's list lives in shared memory)
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -85,7 +99,7 @@ struct BwdCfg {
   static constexpr int META_OFF = BAR_OFF + BAR_BYTES;     // NR step entries
   static constexpr int META_INTS = 24;                     // [0] nvalid [1..8] ids [9..16] keep
   static constexpr int MISC_OFF = META_OFF + NR * META_INTS * 4;
-  static constexpr int MISC_BYTES = 64;                    // tmem base, abort, total, counts[8]
+  static constexpr int MISC_BYTES = 128;                   // tmem base, abort, total, counts[warps]
   static constexpr int STAGE_OFF = MISC_OFF + MISC_BYTES;  // 2 x (128 LSE + 128 D) floats
   static constexpr int STAGE_BYTES = 2 * 2 * 128 * 4;
   static constexpr int BM_OFF = STAGE_OFF + STAGE_BYTES;   // q-block bitmaps (dQ kernel)
@@ -158,12 +172,14 @@ __device__ __forceinline__ void zero_rows(__nv_bfloat16* g, long long bh, int t0
   }
 }
 
-// Store one 128-row accumulator row (this thread's TMEM lane) as bf16, times `mul`.
-template <int D>
+// Store NC columns of one accumulator row (this thread's TMEM lane) as bf16,
+// times `mul`.
+template <int NC>
 __device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bfloat16* dst,
                                               bool store) {
+  static_assert(NC % 32 == 0, "32-column loads");
 #pragma unroll 1
-  for (int c = 0; c < D / 32; ++c) {
+  for (int c = 0; c < NC / 32; ++c) {
     uint32_t r[32];
     tmem_ld32(taddr + c * 32, r);
     tmem_wait_ld();
@@ -251,9 +267,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&ring_free[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, kBwdEltWarps);
     mbar_init(acc_done, 1);
-    mbar_init(stage_bar, 4);
+    mbar_init(stage_bar, kBwdEltWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -363,11 +379,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // dV += P^T dO, dK += dS^T Q (M = 128 keys, N = D, K = 128 queries)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(t_dv, t_s + kk * 8, d_do_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
+          mma_ts(t_dv, t_s + packed_col(kk * 16), d_do_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
                  idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(t_dk, t_dp + kk * 8, d_q_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
+          mma_ts(t_dk, t_dp + packed_col(kk * 16), d_q_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
                  idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&ring_free[slot]);
       }
@@ -385,12 +401,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ================================================================ P^T, dS^T, epilogue
+    // warp (q, part): TMEM lane quarter q = warp % 4, query columns
+    // [part * kBwdCols, part * kBwdCols + kBwdCols) of each step
     const int wq = warp & 3;
+    const int part = (warp - 4) >> 2;
+    const int cbase = part * kBwdCols;
+    const int sbase = cbase / BLK;                // first q slot of this part
     const int u = wq * 32 + lane;                 // key row of the tile
     const int key = kt * 128 + u;
     const bool key_ok = key < p.N;
     const int kvb = u / BLK;                      // its kv-block in the tile
-    const int gt = tid - 128;                     // 0..127 over the four warps
+    const int gt = tid - 128;                     // 0 .. kBwdEltWarps*32 - 1
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const float c2 = p.scale_log2;
     auto warp_arrive = [&](uint64_t* bar) {
@@ -408,7 +429,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // stage LSE (log2 units) and D of the step's 128 queries; a query past N
       // or in an unused slot gets LSE = +inf (P = 0)
       float* st = stage + (s & 1) * 256;
-      {
+      if (gt < 128) {
         const int sl = gt / BLK;
         const int tok = me[1 + sl] * BLK + gt % BLK;
         const bool valid = sl < nvalid && tok < p.N;
@@ -420,35 +441,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int sl = 0; sl < C::G; ++sl)
         if (sl < nvalid && ((me[9 + sl] >> kvb) & 1)) live |= 1u << sl;
       if (!key_ok) live = 0;
+      const uint32_t live_p = live >> sbase;      // bit j: slot sbase + j
       warp_arrive(stage_bar);
       w_ok = mbar_wait(stage_bar, s & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       w_ok = mbar_wait(s_full, s & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
+      const float* stl = st + cbase;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < kBwdCols / 32; ++cc) {
         uint32_t rs[32], rd[32];
-        tmem_ld32(t_lane + C::S_COL + cc * 32, rs);
-        tmem_ld32(t_lane + C::DP_COL + cc * 32, rd);
+        tmem_ld32(t_lane + C::S_COL + cbase + cc * 32, rs);
+        tmem_ld32(t_lane + C::DP_COL + cbase + cc * 32, rd);
         tmem_wait_ld();
         uint32_t pp[16], pd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int c0 = cc * 32 + 2 * e, c1 = c0 + 1;
-          const bool l0 = (live >> (c0 / BLK)) & 1u, l1 = (live >> (c1 / BLK)) & 1u;
-          const float p0 = l0 ? fast_ex2(__uint_as_float(rs[2 * e]) * c2 - st[c0]) : 0.f;
-          const float p1 = l1 ? fast_ex2(__uint_as_float(rs[2 * e + 1]) * c2 - st[c1]) : 0.f;
-          const float d0 = p0 * (__uint_as_float(rd[2 * e]) - st[128 + c0]);
-          const float d1 = p1 * (__uint_as_float(rd[2 * e + 1]) - st[128 + c1]);
+          const int c0 = cc * 32 + 2 * e, c1 = c0 + 1;     // columns within the part
+          const bool l0 = (live_p >> (c0 / BLK)) & 1u, l1 = (live_p >> (c1 / BLK)) & 1u;
+          const float p0 = l0 ? fast_ex2(__uint_as_float(rs[2 * e]) * c2 - stl[c0]) : 0.f;
+          const float p1 = l1 ? fast_ex2(__uint_as_float(rs[2 * e + 1]) * c2 - stl[c1]) : 0.f;
+          const float d0 = p0 * (__uint_as_float(rd[2 * e]) - stl[128 + c0]);
+          const float d1 = p1 * (__uint_as_float(rd[2 * e + 1]) - stl[128 + c1]);
           __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
           __nv_bfloat162 hd = __floats2bfloat162_rn(d0, d1);
           pp[e] = *reinterpret_cast<uint32_t*>(&hp);
           pd[e] = *reinterpret_cast<uint32_t*>(&hd);
         }
-        // bf16 pairs over the fp32 columns already read: queries 32cc.. -> columns 16cc..
-        tmem_st16(t_lane + C::S_COL + cc * 16, pp);
-        tmem_st16(t_lane + C::DP_COL + cc * 16, pd);
+        // bf16 pairs into the first half of this part's columns, over fp32
+        // columns this warp has already read
+        tmem_st16(t_lane + C::S_COL + packed_col(cbase + cc * 32), pp);
+        tmem_st16(t_lane + C::DP_COL + packed_col(cbase + cc * 32), pd);
       }
       tmem_wait_st();
       warp_arrive(p_full);
@@ -459,9 +483,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      const long long row = ((long long)bh * p.N + key) * D;
-      store_acc_row<D>(t_lane + C::ACC0_COL, 1.0f, p.dv + row, key_ok);
-      store_acc_row<D>(t_lane + C::ACC1_COL, p.scale, p.dk + row, key_ok);
+      constexpr int NC = D / kBwdParts;           // accumulator columns per part
+      const long long row = ((long long)bh * p.N + key) * D + part * NC;
+      store_acc_row<NC>(t_lane + C::ACC0_COL + part * NC, 1.0f, p.dv + row, key_ok);
+      store_acc_row<NC>(t_lane + C::ACC1_COL + part * NC, p.scale, p.dk + row, key_ok);
     } else {
       record_error(BSA_ERR_TIMEOUT);
       *(volatile int*)abort_flag = 1;
@@ -559,7 +584,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&ring_free[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 4);
+    mbar_init(p_full, kBwdEltWarps);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -667,7 +692,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // dQ += dS K (M = 128 queries, N = D, K = 128 keys)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(t_dq, t_s + kk * 8, d_k_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
+          mma_ts(t_dq, t_s + packed_col(kk * 16), d_k_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
                  idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&ring_free[slot]);
       }
@@ -685,7 +710,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ================================================================ dS, epilogue
+    // warp (q, part): TMEM lane quarter q = warp % 4, key columns
+    // [part * kBwdCols, part * kBwdCols + kBwdCols) of each step
+    constexpr int SPP = kBwdCols >= BLK ? kBwdCols / BLK : 1;   // kv slots per part
     const int wq = warp & 3;
+    const int part = (warp - 4) >> 2;
+    const int cbase = part * kBwdCols;
+    const int sbase = cbase / BLK;                // first kv slot of this part
+    const int koff = cbase % BLK;                 // key offset inside that slot's block
     const int r = wq * 32 + lane;                 // query row of the tile
     const int token = qt * 128 + r;
     const bool row_ok = token < p.N;
@@ -706,29 +738,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       const int* me = meta + slot * C::META_INTS;
       const int nvalid = me[0];
-      // kv slots this row keeps, and the valid keys of each (the last block may be partial)
+      // this part's kv slots: kept by this row, and their valid keys (the
+      // last block may be partial)
       uint32_t live = 0;
-      int nk[C::G];
+      int nk[SPP];
 #pragma unroll
-      for (int sl = 0; sl < C::G; ++sl) {
-        if (row_ok && sl < nvalid && ((me[9 + sl] >> qq) & 1)) live |= 1u << sl;
-        nk[sl] = min(BLK, p.N - me[1 + sl] * BLK);
+      for (int j = 0; j < SPP; ++j) {
+        const int sl = sbase + j;
+        if (row_ok && sl < nvalid && ((me[9 + sl] >> qq) & 1)) live |= 1u << j;
+        nk[j] = min(BLK, p.N - me[1 + sl] * BLK);
       }
       w_ok = mbar_wait(s_full, s & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < kBwdCols / 32; ++cc) {
         uint32_t rs[32], rd[32];
-        tmem_ld32(t_lane + C::S_COL + cc * 32, rs);
-        tmem_ld32(t_lane + C::DP_COL + cc * 32, rd);
+        tmem_ld32(t_lane + C::S_COL + cbase + cc * 32, rs);
+        tmem_ld32(t_lane + C::DP_COL + cbase + cc * 32, rd);
         tmem_wait_ld();
         uint32_t pd[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int c0 = cc * 32 + 2 * e, c1 = c0 + 1;
-          const bool l0 = ((live >> (c0 / BLK)) & 1u) && (c0 % BLK) < nk[c0 / BLK];
-          const bool l1 = ((live >> (c1 / BLK)) & 1u) && (c1 % BLK) < nk[c1 / BLK];
+          const int c0 = cc * 32 + 2 * e, c1 = c0 + 1;     // columns within the part
+          const bool l0 = ((live >> (c0 / BLK)) & 1u) && koff + (c0 % BLK) < nk[c0 / BLK];
+          const bool l1 = ((live >> (c1 / BLK)) & 1u) && koff + (c1 % BLK) < nk[c1 / BLK];
           const float p0 = l0 ? fast_ex2(__uint_as_float(rs[2 * e]) * c2 - lse2) : 0.f;
           const float p1 = l1 ? fast_ex2(__uint_as_float(rs[2 * e + 1]) * c2 - lse2) : 0.f;
           const float d0 = p0 * (__uint_as_float(rd[2 * e]) - dlt);
@@ -736,8 +770,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           __nv_bfloat162 hd = __floats2bfloat162_rn(d0, d1);
           pd[e] = *reinterpret_cast<uint32_t*>(&hd);
         }
-        // dS (bf16 pairs) over the S columns already read
-        tmem_st16(t_lane + C::S_COL + cc * 16, pd);
+        // dS (bf16 pairs) into the first half of this part's columns
+        tmem_st16(t_lane + C::S_COL + packed_col(cbase + cc * 32), pd);
       }
       tmem_wait_st();
       warp_arrive(p_full);
@@ -748,7 +782,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     if (ok) {
       tc_fence_after();
-      store_acc_row<D>(t_lane + C::ACC0_COL, p.scale, p.dq + ((long long)bh * p.N + token) * D, row_ok);
+      constexpr int NC = D / kBwdParts;
+      store_acc_row<NC>(t_lane + C::ACC0_COL + part * NC, p.scale,
+                        p.dq + ((long long)bh * p.N + token) * D + part * NC, row_ok);
     } else {
       record_error(BSA_ERR_TIMEOUT);
       *(volatile int*)abort_flag = 1;
