@@ -70,9 +70,12 @@ def pattern_row(pattern: int, i: int, nb: int, n: int, blk: int, band_w: int, fr
         for f in range(f_lo, f_hi + 1):
             keep |= (lo <= f * S + band_w * blk) & (hi >= f * S - band_w * blk)
     elif pattern == STRIPE:
-        # the first stripe token at or after uj_lo lies in the block
+        # the first stripe token at or after uj_lo lies in the block (there is
+        # none when a frame has no stripe tokens)
         f = uj_lo // S
         keep = ((uj_lo - f * S) < stripe_blocks * blk) | ((f + 1) * S <= uj_hi)
+        if stripe_blocks <= 0:
+            keep = np.zeros(nb, dtype=bool)
     elif pattern == TILE3D:
         fi_lo, fi_hi = ti_lo // S, ti_hi // S
         fj_lo, fj_hi = uj_lo // S, uj_hi // S

@@ -16,6 +16,7 @@ CASES = [
     (70, 16, 30, 0, -2, 2, 1, 2),
     (64, 4, 16, 2, 0, 0, 3, 1),
     (50, 7, 13, 1, -3, 3, 1, 1),
+    (90, 8, 21, 1, -1, 1, 0, 0),      # no stripe tokens: frame starts inside blocks
 ]
 
 
