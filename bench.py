@@ -297,8 +297,9 @@ class Layer:
                                dtype=torch.uint8, device=dev)
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-        # kernels per step: pool, select, scan, expand (ASA) or pattern + scan
-        self.launches = (4 if w.source == "asa" else 3) + 1
+        # kernels per step: pool and select (ASA) or pattern count, scan and
+        # write; then the forward
+        self.launches = (2 if w.source == "asa" else 3) + 1
 
     def mask(self):
         w, b = self.w, self.bsa
@@ -383,8 +384,10 @@ def layer_summary(layer: Layer, t: dict, pk: dict, steps: int) -> dict:
 
 
 def time_backward(bsa, layer: Layer, flops: float, pk: dict, iters: int = 10, warmup: int = 3):
-    """bsa_backward on the layer's mask, O and LSE for a seeded dO (CUDA events,
-    median of `iters` calls).  Flops at the usual 2.5x the forward's block flops."""
+    """The training path's backward (bsa_backward with the forward's rounding
+    residual, as the autograd node runs it) on the layer's mask, O and LSE for a
+    seeded dO (CUDA events, median of `iters` calls).  Flops at the usual 2.5x
+    the forward's block flops."""
     q, k, v, w = layer.q, layer.k, layer.v, layer.w
     B, H, N, d = q.shape
     g = torch.Generator(device=q.device).manual_seed(5)
@@ -392,10 +395,13 @@ def time_backward(bsa, layer: Layer, flops: float, pk: dict, iters: int = 10, wa
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(max(bsa.backward_workspace_size(B, H, N, d, w.blk), 4), dtype=torch.uint8,
                      device=q.device)
+    res = torch.empty_like(q)
+    bsa.bsa_forward_into(q, k, v, w.blk, layer.row_ptr, layer.col_idx, layer.o, layer.lse,
+                         workspace=layer.fws, o_residual=res)
 
     def call():
         bsa.bsa_backward_into(q, k, v, layer.o, dout, layer.lse, w.blk, layer.row_ptr,
-                              layer.col_idx, dq, dk, dv, 0.0, ws)
+                              layer.col_idx, dq, dk, dv, 0.0, ws, o_residual=res)
     for _ in range(warmup):
         call()
     check_status(bsa, "after backward warm-up")
@@ -412,7 +418,7 @@ def time_backward(bsa, layer: Layer, flops: float, pk: dict, iters: int = 10, wa
     tf = 2.5 * flops / (ms * 1e-3) / 1e12
     return {"workload": w.name, "ms_backward": ms, "tflops_2p5x": tf,
             "frac": tf / float(pk["bf16_tflops"]), "flop_convention": "2.5x forward block flops",
-            "iters": iters}
+            "d_from": "fp32 O (forward rounding residual)", "iters": iters}
 
 
 def run_gpu(args, rank, world, local):

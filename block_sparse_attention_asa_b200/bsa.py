@@ -48,7 +48,11 @@ _SIGNATURES = {
     "bsa_forward_workspace_size": (_c_size, [_c_int] * 5),
     "bsa_forward": (_c_int, [_vp, _vp, _vp] + [_c_int] * 5 + [_vp, _vp, _c_float, _vp, _vp, _vp,
                                                               _c_size, _vp]),
+    "bsa_forward_residual": (_c_int, [_vp, _vp, _vp] + [_c_int] * 5 + [_vp, _vp, _c_float, _vp, _vp,
+                                                                       _vp, _vp, _c_size, _vp]),
     "bsa_backward_workspace_size": (_c_size, [_c_int] * 5),
+    "bsa_backward_residual": (_c_int, [_vp] * 7 + [_c_int] * 5 + [_vp, _vp, _c_float, _vp, _vp,
+                                                                  _vp, _vp, _c_size, _vp]),
     "bsa_backward": (_c_int, [_vp] * 6 + [_c_int] * 5 + [_vp, _vp, _c_float, _vp, _vp, _vp, _vp,
                                                           _c_size, _vp]),
     "bsa_validate_csr_host": (_c_int, [_vp, _vp, _c_i64, _c_int, _c_i64, _vp]),
@@ -249,19 +253,28 @@ def forward_workspace_size(B: int, H: int, N: int, d: int, blk: int) -> int:
 
 
 def bsa_forward_into(q, k, v, blk, row_ptr, col_idx, o, lse=None, softmax_scale=0.0,
-                     workspace=None, stream=None):
+                     workspace=None, stream=None, o_residual=None):
     B, H, N, d = _shape(q)
     lib = load()
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = lib.bsa_forward(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, blk, _ptr(row_ptr), _ptr(col_idx),
-                         softmax_scale, _ptr(o), _ptr(lse), _ptr(workspace), ws_bytes,
-                         _stream(stream))
-    _check(rc, "bsa_forward")
+    if o_residual is None:
+        rc = lib.bsa_forward(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, blk, _ptr(row_ptr),
+                             _ptr(col_idx), softmax_scale, _ptr(o), _ptr(lse), _ptr(workspace),
+                             ws_bytes, _stream(stream))
+        _check(rc, "bsa_forward")
+        return
+    rc = lib.bsa_forward_residual(_ptr(q), _ptr(k), _ptr(v), B, H, N, d, blk, _ptr(row_ptr),
+                                  _ptr(col_idx), softmax_scale, _ptr(o), _ptr(lse),
+                                  _ptr(o_residual), _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "bsa_forward_residual")
 
 
 def bsa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blk: int, row_ptr: torch.Tensor,
-                col_idx: torch.Tensor, softmax_scale: float = 0.0, stream=None):
-    """(O bf16 [B,H,N,d], LSE fp32 [B,H,N]) of attention over the CSR's kept blocks."""
+                col_idx: torch.Tensor, softmax_scale: float = 0.0, stream=None,
+                residual: bool = False):
+    """(O bf16 [B,H,N,d], LSE fp32 [B,H,N]) of attention over the CSR's kept blocks;
+    with residual=True also O's bf16 rounding residual (O + residual carries the
+    fp32 O), for bsa_backward's o_residual."""
     _need_cuda(q, k, v, row_ptr)
     B, H, N, d = _shape(q)
     o = torch.empty_like(q)
@@ -270,8 +283,9 @@ def bsa_forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, blk: int, row
     ws = torch.empty(ws_n, dtype=torch.uint8, device=q.device) if ws_n else None
     if col_idx.numel() == 0:
         col_idx = torch.zeros(1, dtype=torch.int32, device=q.device)
-    bsa_forward_into(q, k, v, blk, row_ptr, col_idx, o, lse, softmax_scale, ws, stream)
-    return o, lse
+    res = torch.empty_like(q) if residual else None
+    bsa_forward_into(q, k, v, blk, row_ptr, col_idx, o, lse, softmax_scale, ws, stream, res)
+    return (o, lse, res) if residual else (o, lse)
 
 
 # ----------------------------------------------------------------------------- backward
@@ -280,20 +294,29 @@ def backward_workspace_size(B: int, H: int, N: int, d: int, blk: int) -> int:
 
 
 def bsa_backward_into(q, k, v, o, dout, lse, blk, row_ptr, col_idx, dq, dk, dv,
-                      softmax_scale=0.0, workspace=None, stream=None):
+                      softmax_scale=0.0, workspace=None, stream=None, o_residual=None):
     B, H, N, d = _shape(q)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = load().bsa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), B, H, N,
-                             d, blk, _ptr(row_ptr), _ptr(col_idx), softmax_scale, _ptr(dq),
-                             _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _stream(stream))
-    _check(rc, "bsa_backward")
+    if o_residual is None:
+        rc = load().bsa_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), B, H,
+                                 N, d, blk, _ptr(row_ptr), _ptr(col_idx), softmax_scale, _ptr(dq),
+                                 _ptr(dk), _ptr(dv), _ptr(workspace), ws_bytes, _stream(stream))
+        _check(rc, "bsa_backward")
+        return
+    rc = load().bsa_backward_residual(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(o_residual),
+                                      _ptr(dout), _ptr(lse), B, H, N, d, blk, _ptr(row_ptr),
+                                      _ptr(col_idx), softmax_scale, _ptr(dq), _ptr(dk), _ptr(dv),
+                                      _ptr(workspace), ws_bytes, _stream(stream))
+    _check(rc, "bsa_backward_residual")
 
 
 def bsa_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
                  dout: torch.Tensor, lse: torch.Tensor, blk: int, row_ptr: torch.Tensor,
-                 col_idx: torch.Tensor, softmax_scale: float = 0.0, stream=None):
+                 col_idx: torch.Tensor, softmax_scale: float = 0.0, stream=None,
+                 o_residual: Optional[torch.Tensor] = None):
     """(dQ, dK, dV) bf16 [B,H,N,d] of attention over the CSR's kept blocks for the
-    incoming gradient dout; o and lse are bsa_forward's outputs for the same call."""
+    incoming gradient dout; o and lse are bsa_forward's outputs for the same call
+    (o_residual: its residual output, so that D comes from the fp32 O)."""
     _need_cuda(q, k, v, o, dout, lse, row_ptr)
     B, H, N, d = _shape(q)
     for t in (k, v, o, dout):
@@ -306,30 +329,34 @@ def bsa_backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Ten
                      device=q.device)
     if col_idx.numel() == 0:
         col_idx = torch.zeros(1, dtype=torch.int32, device=q.device)
+    if o_residual is not None and (tuple(o_residual.shape) != (B, H, N, d) or
+                                   o_residual.dtype != torch.bfloat16):
+        raise ValueError("o_residual must match q (bf16 [B, H, N, d])")
     bsa_backward_into(q, k, v, o, dout, lse, blk, row_ptr, col_idx, dq, dk, dv, softmax_scale, ws,
-                      stream)
+                      stream, o_residual)
     return dq, dk, dv
 
 
 class _BlockSparseAttention(torch.autograd.Function):
     """bsa_forward / bsa_backward as one autograd node.  The mask is a constant
     of the step and only O is returned, so nothing downstream can depend on an
-    undifferentiated LSE."""
+    undifferentiated LSE.  The forward keeps O's rounding residual for the
+    backward, so that D comes from the fp32 O."""
 
     @staticmethod
     def forward(ctx, q, k, v, blk, row_ptr, col_idx, softmax_scale):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        o, lse = bsa_forward(q, k, v, blk, row_ptr, col_idx, softmax_scale)
-        ctx.save_for_backward(q, k, v, o, lse, row_ptr, col_idx)
+        o, lse, res = bsa_forward(q, k, v, blk, row_ptr, col_idx, softmax_scale, residual=True)
+        ctx.save_for_backward(q, k, v, o, lse, res, row_ptr, col_idx)
         ctx.blk = blk
         ctx.softmax_scale = softmax_scale
         return o
 
     @staticmethod
     def backward(ctx, dout):
-        q, k, v, o, lse, row_ptr, col_idx = ctx.saved_tensors
+        q, k, v, o, lse, res, row_ptr, col_idx = ctx.saved_tensors
         dq, dk, dv = bsa_backward(q, k, v, o, dout.contiguous().to(torch.bfloat16), lse, ctx.blk,
-                                  row_ptr, col_idx, ctx.softmax_scale)
+                                  row_ptr, col_idx, ctx.softmax_scale, o_residual=res)
         return dq, dk, dv, None, None, None, None
 
 

@@ -21,8 +21,12 @@
 //                       reductions -> selection bitmap and count.
 //   asa_select_generic_kernel   any nb: the same arithmetic with the row kept in
 //                       shared memory and a radix select on the 64-bit key.
-//   csr_scan_kernel     counts -> row_ptr.
-//   asa_expand_kernel   bitmaps -> ascending col_idx.
+//                       Both select kernels then write the CSR themselves: a
+//                       CTA takes its rows in the order of a ticket counter,
+//                       publishes its rows' total, finds the total of all
+//                       earlier rows by a decoupled look-back over the earlier
+//                       CTAs' published totals, writes its row_ptr entries and
+//                       expands its bitmaps into ascending col_idx.
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -43,7 +47,15 @@ constexpr int kPoolWarps = 4;
 template <int D, int BLK>
 __global__ void __launch_bounds__(kPoolWarps * 32) asa_pool_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-    float* __restrict__ qbar, float* __restrict__ kbarT, int BH, int N, int nb, int kt_ld) {
+    float* __restrict__ qbar, float* __restrict__ kbarT, int BH, int N, int nb, int kt_ld,
+    unsigned long long* __restrict__ scan_flags, unsigned int* __restrict__ scan_ticket,
+    int n_flags) {
+  // the select kernel's look-back state starts at zero (the grid has more CTAs
+  // than there are flags)
+  if (threadIdx.x == 0) {
+    if (blockIdx.x < static_cast<unsigned>(n_flags)) scan_flags[blockIdx.x] = 0ull;
+    if (blockIdx.x == 0) *scan_ticket = 0u;
+  }
   constexpr int blk = BLK;
   constexpr int LPR = D / 8;          // lanes per row
   constexpr int RPS = 32 / LPR;       // rows per warp step
@@ -108,7 +120,13 @@ struct SelectParams {
   const float* qbar;      // [BH*nb, D]
   const float* kbarT;     // [BH, D, kt_ld]: k̄ transposed, rows padded to kt_ld
   uint32_t* bitmaps;      // [BH*nb, nbw]
-  int32_t* row_ptr;       // counts go to row_ptr[r+1]
+  int32_t* row_ptr;       // [BH*nb + 1]
+  int32_t* col_idx;       // [capacity]
+  long long capacity;
+  unsigned long long* scan_flags;   // [CTAs]: per CTA (total << 2) | state, zeroed before launch
+  unsigned int* scan_ticket;        // CTA order, zeroed before launch
+  unsigned long long wait_ns;       // bound on the look-back wait
+  int groups;             // CTAs per (b, h)
   int nb, nbw, rows_per_cta, nb_pad, kt_ld;
   int dk;                 // asa_select_kernel: k̄ᵀ rows per cp.async stage
   int mode, topk, cap, keep_diag, n_sink;
@@ -257,6 +275,90 @@ __device__ int mass_count(const float* pr, int nb, float tau, int limit, unsigne
   return limit;
 }
 
+// The CTA that took ticket `lin` and owns rows [i0, i0 + nrow) of (b, h) = bh:
+// its rows' counts (cnt, shared memory) are published, the total of every
+// earlier row is found by a decoupled look-back, then row_ptr is written and
+// the row bitmaps (already in global memory, written by this CTA) are expanded
+// into ascending block ids.  Flag word per CTA: (total << 2) | state, state 1 =
+// the CTA's own total, 2 = the total through this CTA.  A CTA waits only for
+// CTAs with smaller tickets, which started before it, so the wait ends; it is
+// bounded all the same (BSA_ERR_TIMEOUT).
+__device__ __forceinline__ void csr_write_rows(const SelectParams& p, int lin, int bh, int i0,
+                                               int nrow, const int* cnt, long long* s_base) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  __syncthreads();   // counts and bitmaps of every row of the CTA are written
+  if (warp == 0) {
+    long long agg = 0;
+    for (int r = lane; r < nrow; r += 32) agg += cnt[r];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) agg += __shfl_xor_sync(0xffffffffu, agg, o);
+    volatile unsigned long long* fl = p.scan_flags;
+    if (lane == 0) atomicExch(p.scan_flags + lin, (static_cast<unsigned long long>(agg) << 2) |
+                                                      (lin == 0 ? 2ull : 1ull));
+    long long prefix = 0;
+    int j = lin - 1;   // nearest CTA not yet accounted for
+    const uint64_t t0 = global_ns();
+    while (j >= 0) {
+      const int idx = j - lane;
+      const unsigned long long f = idx >= 0 ? fl[idx] : 2ull;   // before CTA 0: total 0
+      const unsigned st = static_cast<unsigned>(f & 3ull);
+      const unsigned incl = __ballot_sync(0xffffffffu, st == 2u);
+      const unsigned zero = __ballot_sync(0xffffffffu, st == 0u);
+      const int stop = incl ? __ffs(incl) - 1 : 31;           // last lane to add
+      const unsigned upto = stop == 31 ? 0xffffffffu : ((2u << stop) - 1u);
+      if (zero & upto) {
+        if (global_ns() - t0 > p.wait_ns) {
+          if (lane == 0) record_error(BSA_ERR_TIMEOUT);
+          break;
+        }
+        continue;
+      }
+      long long v = lane <= stop ? static_cast<long long>(f >> 2) : 0;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      prefix += v;
+      if (incl) break;
+      j -= 32;
+    }
+    if (lin > 0 && lane == 0)
+      atomicExch(p.scan_flags + lin, (static_cast<unsigned long long>(prefix + agg) << 2) | 2ull);
+    if (lane == 0) *s_base = prefix;
+  }
+  __syncthreads();
+  const long long base = *s_base;
+  if (lin == 0 && tid == 0) p.row_ptr[0] = 0;
+  // one warp per row: its end in row_ptr, its blocks in ascending order
+  for (int rr = warp; rr < nrow; rr += kSelWarps) {
+    long long before = 0;
+    for (int r = 0; r < rr; ++r) before += cnt[r];
+    long long pos = base + before;
+    const long long row = (long long)bh * p.nb + i0 + rr;
+    if (lane == 0) {
+      const long long end = pos + cnt[rr];
+      if (end > 0x7fffffffLL) record_error(BSA_ERR_CAPACITY);
+      p.row_ptr[row + 1] = static_cast<int32_t>(end > 0x7fffffffLL ? 0x7fffffffLL : end);
+    }
+    const uint32_t* bmr = p.bitmaps + row * p.nbw;
+    for (int w0 = 0; w0 < p.nbw; w0 += 32) {
+      const int wd = w0 + lane;
+      uint32_t word = wd < p.nbw ? bmr[wd] : 0u;
+      const int c = __popc(word);
+      const int incl = warp_incl_scan(c);
+      long long at = pos + incl - c;
+      while (word) {
+        const int bit = __ffs(word) - 1;
+        word &= word - 1;
+        if (at < p.capacity)
+          p.col_idx[at] = wd * 32 + bit;
+        else
+          record_error(BSA_ERR_CAPACITY);
+        ++at;
+      }
+      pos += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(256) asa_select_generic_kernel(const SelectParams p) {
   extern __shared__ __align__(16) unsigned char sel_smem[];
@@ -267,9 +369,15 @@ __global__ void __launch_bounds__(256) asa_select_generic_kernel(const SelectPar
   unsigned int* hist = reinterpret_cast<unsigned int*>(sc + (size_t)R * p.nb_pad);  // [8][256]
   unsigned long long* buf =
       reinterpret_cast<unsigned long long*>(hist + kSelWarps * 256);  // [8][64]
+  __shared__ int s_cnt[64];
+  __shared__ long long s_base;
+  __shared__ int s_lin;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.y, i0 = blockIdx.x * R;
+  if (tid == 0) s_lin = static_cast<int>(atomicAdd(p.scan_ticket, 1u));
+  __syncthreads();
+  const int lin = s_lin;
+  const int bh = lin / p.groups, i0 = (lin % p.groups) * R;
   const int nrow = min(R, p.nb - i0);
   const float* qrow = p.qbar + ((long long)bh * p.nb + i0) * D;
   const float* kbh = p.kbarT + (long long)bh * D * p.kt_ld;
@@ -343,9 +451,10 @@ __global__ void __launch_bounds__(256) asa_select_generic_kernel(const SelectPar
       if (lane == 0) dst[wd] = word;
       cnt += __popc(word);
     }
-    if (lane == 0) p.row_ptr[r + 1] = cnt;
+    if (lane == 0) s_cnt[rr] = cnt;
     __syncwarp();
   }
+  csr_write_rows(p, lin, bh, i0, nrow, s_cnt, &s_base);
 }
 
 // ------------------------------------------------------------------ select, registers
@@ -446,7 +555,7 @@ __device__ __forceinline__ unsigned keep_bits(const unsigned (&u)[NPL], int nb, 
 // the row's bitmap words and count.
 template <int NPL>
 __device__ __forceinline__ void select_row_regs(const float* srow, int i, long long row,
-                                                const SelectParams& p) {
+                                                const SelectParams& p, int* cnt_out) {
   const int lane = threadIdx.x & 31;
   const int nb = p.nb;
   float v[NPL];
@@ -524,7 +633,7 @@ __device__ __forceinline__ void select_row_regs(const float* srow, int i, long l
     cnt += __popc(w);
   }
   if (lane < p.nbw) p.bitmaps[row * p.nbw + lane] = myword;
-  if (lane == 0) p.row_ptr[row + 1] = cnt;
+  if (lane == 0) *cnt_out = cnt;
 }
 
 // Tile shape of asa_select_kernel for nb in (128 (NCB-1), 128 NCB], NCB <= 8.
@@ -556,8 +665,14 @@ __global__ void __launch_bounds__(256, NCB > 4 ? 2 : 3) asa_select_kernel(const 
   extern __shared__ __align__(16) float sel_f[];
   float* qs = sel_f;
   float* ka = sel_f + D * R;
+  __shared__ int s_cnt[R];
+  __shared__ long long s_base;
+  __shared__ int s_lin;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int bh = blockIdx.y, i0 = blockIdx.x * R;
+  if (tid == 0) s_lin = static_cast<int>(atomicAdd(p.scan_ticket, 1u));
+  __syncthreads();
+  const int lin = s_lin;
+  const int bh = lin / p.groups, i0 = (lin % p.groups) * R;
   const int nrow = min(R, p.nb - i0);
   const int rt = warp / ncb, ct = warp - rt * ncb;
   const bool active = warp < (R >> 3) * ncb && rt * 8 < nrow;
@@ -634,38 +749,9 @@ __global__ void __launch_bounds__(256, NCB > 4 ? 2 : 3) asa_select_kernel(const 
   }
   __syncthreads();
   for (int rr = warp; rr < nrow; rr += kSelWarps)
-    select_row_regs<NPL>(ka + rr * nb_pad, i0 + rr, (long long)bh * p.nb + i0 + rr, p);
-}
-
-// ------------------------------------------------------------------ expand
-// One warp per row: set bits of the row's bitmap -> ascending block ids.
-__global__ void __launch_bounds__(256) asa_expand_kernel(const uint32_t* __restrict__ bitmaps,
-                                                         const int32_t* __restrict__ row_ptr,
-                                                         int32_t* __restrict__ col_idx,
-                                                         long long capacity, long long rows,
-                                                         int nbw) {
-  const int lane = threadIdx.x & 31;
-  const long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (r >= rows) return;
-  long long pos = row_ptr[r];
-  const uint32_t* bmr = bitmaps + r * nbw;
-  for (int w0 = 0; w0 < nbw; w0 += 32) {
-    const int wd = w0 + lane;
-    uint32_t word = wd < nbw ? bmr[wd] : 0u;
-    const int c = __popc(word);
-    const int incl = warp_incl_scan(c);
-    long long at = pos + incl - c;
-    while (word) {
-      const int bit = __ffs(word) - 1;
-      word &= word - 1;
-      if (at < capacity)
-        col_idx[at] = wd * 32 + bit;
-      else
-        record_error(BSA_ERR_CAPACITY);
-      ++at;
-    }
-    pos += __shfl_sync(0xffffffffu, incl, 31);
-  }
+    select_row_regs<NPL>(ka + rr * nb_pad, i0 + rr, (long long)bh * p.nb + i0 + rr, p,
+                         &s_cnt[rr]);
+  csr_write_rows(p, lin, bh, i0, nrow, s_cnt, &s_base);
 }
 
 }  // namespace bsa

@@ -112,7 +112,7 @@ int sm_count() {
 template <int D, int BLK>
 int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
                const int32_t* row_ptr, const int32_t* col_idx, float scale, void* o, float* lse,
-               int* item_counter, cudaStream_t stream) {
+               void* o_res, int* item_counter, cudaStream_t stream) {
   using C = FwdCfg<D, BLK>;
   const int nb = (N + BLK - 1) / BLK;
   const int nbw = (nb + 31) / 32;
@@ -137,6 +137,7 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
+  p.o_res = static_cast<__nv_bfloat16*>(o_res);
   p.wait_ns = kWaitNs;
   p.item_counter = item_counter;
   const int sms = sm_count();
@@ -150,12 +151,12 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
 template <int D>
 int launch_fwd_blk(int blk, const void* q, const void* k, const void* v, int B, int H, int N,
                    const int32_t* rp, const int32_t* ci, float scale, void* o, float* lse,
-                   int* ctr, cudaStream_t s) {
+                   void* o_res, int* ctr, cudaStream_t s) {
   switch (blk) {
-    case 16: return launch_fwd<D, 16>(q, k, v, B, H, N, rp, ci, scale, o, lse, ctr, s);
-    case 32: return launch_fwd<D, 32>(q, k, v, B, H, N, rp, ci, scale, o, lse, ctr, s);
-    case 64: return launch_fwd<D, 64>(q, k, v, B, H, N, rp, ci, scale, o, lse, ctr, s);
-    case 128: return launch_fwd<D, 128>(q, k, v, B, H, N, rp, ci, scale, o, lse, ctr, s);
+    case 16: return launch_fwd<D, 16>(q, k, v, B, H, N, rp, ci, scale, o, lse, o_res, ctr, s);
+    case 32: return launch_fwd<D, 32>(q, k, v, B, H, N, rp, ci, scale, o, lse, o_res, ctr, s);
+    case 64: return launch_fwd<D, 64>(q, k, v, B, H, N, rp, ci, scale, o, lse, o_res, ctr, s);
+    case 128: return launch_fwd<D, 128>(q, k, v, B, H, N, rp, ci, scale, o, lse, o_res, ctr, s);
   }
   return BSA_ERR_UNSUPPORTED;
 }
@@ -165,7 +166,7 @@ int launch_fwd_blk(int blk, const void* q, const void* k, const void* v, int B, 
 // each part starting on a 256-byte boundary.
 struct AsaLayout {
   long long nb, nbw, rows, kt_ld;
-  size_t qbar_off, kbar_off, bitmap_off, total;
+  size_t qbar_off, kbar_off, bitmap_off, scan_off, total;
 };
 
 AsaLayout asa_layout(int B, int H, int N, int d, int blk) {
@@ -178,7 +179,10 @@ AsaLayout asa_layout(int B, int H, int N, int d, int blk) {
   L.qbar_off = 0;
   L.kbar_off = up((size_t)L.rows * d * sizeof(float));
   L.bitmap_off = L.kbar_off + up((size_t)B * H * d * L.kt_ld * sizeof(float));
-  L.total = L.bitmap_off + up((size_t)L.rows * L.nbw * sizeof(uint32_t));
+  // the select kernels' look-back state: a ticket, then one flag word per CTA
+  // (at most one CTA per row)
+  L.scan_off = L.bitmap_off + up((size_t)L.rows * L.nbw * sizeof(uint32_t));
+  L.total = L.scan_off + 256 + up((size_t)L.rows * sizeof(unsigned long long));
   return L;
 }
 
@@ -200,9 +204,10 @@ int launch_select_regs(bsa::SelectParams sp, int BH, cudaStream_t stream) {
   sp.nb_pad = T::NB_PAD;
   sp.rows_per_cta = T::R;
   sp.dk = T::DK;
+  sp.groups = static_cast<int>(ceil_div(sp.nb, T::R));
   static DeviceFlags done;
   if (!allow_smem(bsa::asa_select_kernel<D, NCB>, T::SMEM, done)) return BSA_ERR_CUDA;
-  dim3 grid(ceil_div(sp.nb, T::R), BH);
+  const dim3 grid(static_cast<unsigned>((long long)sp.groups * BH));
   bsa::asa_select_kernel<D, NCB><<<grid, 256, T::SMEM, stream>>>(sp);
   return check_launch() ? BSA_ERR_CUDA : BSA_OK;
 }
@@ -219,7 +224,10 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
   float* qbar = reinterpret_cast<float*>(base + L.qbar_off);
   float* kbarT = reinterpret_cast<float*>(base + L.kbar_off);
   uint32_t* bitmaps = reinterpret_cast<uint32_t*>(base + L.bitmap_off);
-  // 1. pooling
+  auto* scan_ticket = reinterpret_cast<unsigned int*>(base + L.scan_off);
+  auto* scan_flags = reinterpret_cast<unsigned long long*>(base + L.scan_off + 256);
+  const int n_flags = static_cast<int>(L.rows);
+  // 1. pooling (also zeroes the select kernel's look-back state)
   {
     const long long units = 2LL * BH * nb;
     const auto* qq = static_cast<const __nv_bfloat16*>(q);
@@ -227,10 +235,10 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
     const int ld = static_cast<int>(L.kt_ld);
     const dim3 g(static_cast<unsigned>(units)), b(bsa::kPoolWarps * 32);
     switch (blk) {
-      case 16: bsa::asa_pool_kernel<D, 16><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld); break;
-      case 32: bsa::asa_pool_kernel<D, 32><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld); break;
-      case 64: bsa::asa_pool_kernel<D, 64><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld); break;
-      case 128: bsa::asa_pool_kernel<D, 128><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld); break;
+      case 16: bsa::asa_pool_kernel<D, 16><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld, scan_flags, scan_ticket, n_flags); break;
+      case 32: bsa::asa_pool_kernel<D, 32><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld, scan_flags, scan_ticket, n_flags); break;
+      case 64: bsa::asa_pool_kernel<D, 64><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld, scan_flags, scan_ticket, n_flags); break;
+      case 128: bsa::asa_pool_kernel<D, 128><<<g, b, 0, stream>>>(qq, kk, qbar, kbarT, BH, N, nb, ld, scan_flags, scan_ticket, n_flags); break;
       default: return BSA_ERR_UNSUPPORTED;
     }
     if (check_launch()) return BSA_ERR_CUDA;
@@ -242,6 +250,11 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
     sp.kbarT = kbarT;
     sp.bitmaps = bitmaps;
     sp.row_ptr = row_ptr;
+    sp.col_idx = col_idx;
+    sp.capacity = cap_entries;
+    sp.scan_flags = scan_flags;
+    sp.scan_ticket = scan_ticket;
+    sp.wait_ns = kWaitNs;
     sp.nb = nb;
     sp.nbw = nbw;
     sp.kt_ld = static_cast<int>(L.kt_ld);
@@ -277,19 +290,13 @@ int launch_asa(const void* q, const void* k, int B, int H, int N, int blk, int m
       if (!allow_smem(bsa::asa_select_generic_kernel<D>, 220 * 1024, done)) return BSA_ERR_CUDA;
       sp.rows_per_cta = R;
       sp.nb_pad = nb_pad;
-      dim3 grid(ceil_div(nb, R), BH);
+      sp.groups = static_cast<int>(ceil_div(nb, R));
+      const dim3 grid(static_cast<unsigned>((long long)sp.groups * BH));
       bsa::asa_select_generic_kernel<D><<<grid, 256, smem, stream>>>(sp);
       rc = check_launch() ? BSA_ERR_CUDA : BSA_OK;
     }
-    if (rc != BSA_OK) return rc;
+    return rc;
   }
-  // 3. counts -> row_ptr
-  bsa::csr_scan_kernel<<<1, 1024, 0, stream>>>(row_ptr, static_cast<int>(L.rows));
-  if (check_launch()) return BSA_ERR_CUDA;
-  // 4. bitmaps -> col_idx
-  bsa::asa_expand_kernel<<<ceil_div(L.rows, 8), 256, 0, stream>>>(bitmaps, row_ptr, col_idx,
-                                                                  cap_entries, L.rows, nbw);
-  return check_launch();
 }
 
 // ---- backward launches ---------------------------------------------------------
@@ -563,22 +570,28 @@ int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
   p.H = H;
   p.N = N;
   p.blk = blk;
+  p.lblk = blk == 16 ? 4 : blk == 32 ? 5 : blk == 64 ? 6 : 7;   // blk checked above
   p.nb = (N + blk - 1) / blk;
+  // The kernels compute in 32 bits: band widths above 2^24 tokens and frames
+  // above 2^28 tokens are not supported, and two clamps that change no mask
+  // keep the rest in range (a stripe of nb blocks covers a whole frame; there
+  // are at most N / frame_tokens + 1 frames).
+  if ((long long)band_w * blk > (1LL << 24) || frame_tokens > (1 << 28))
+    return BSA_ERR_UNSUPPORTED;
+  const int frames = N / frame_tokens + 1;
   p.band_w = band_w;
   p.frame_tokens = frame_tokens;
   p.f_lo = f_lo;
   p.f_hi = f_hi;
-  p.stripe_blocks = stripe_blocks;
-  p.tile_global_frames = tile_global_frames;
+  p.stripe_blocks = stripe_blocks < p.nb ? stripe_blocks : p.nb;
+  p.tile_global_frames = tile_global_frames < frames ? tile_global_frames : frames;
   p.row_ptr = row_ptr;
   p.col_idx = col_idx;
   p.capacity = col_capacity;
   cudaStream_t s = as_cuda(stream);
   const long long units = (long long)H * p.nb;
   const long long rows = (long long)B * H * p.nb;
-  bsa::pattern_kernel<false><<<ceil_div(units, 8), 256, 0, s>>>(p);
-  if (check_launch()) return BSA_ERR_CUDA;
-  bsa::csr_scan_kernel<<<1, 1024, 0, s>>>(row_ptr, static_cast<int>(rows));
+  bsa::pattern_rowptr_kernel<<<H, bsa::kPatternScanThreads, 0, s>>>(p);
   if (check_launch()) return BSA_ERR_CUDA;
   if (nnz_out_host) {
     int32_t nnz = 0;
@@ -589,7 +602,7 @@ int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
     *nnz_out_host = nnz;
     if (nnz > col_capacity) return BSA_ERR_CAPACITY;
   }
-  bsa::pattern_kernel<true><<<ceil_div(units, 8), 256, 0, s>>>(p);
+  bsa::pattern_write_kernel<<<ceil_div(units, 8), 256, 0, s>>>(p);
   return check_launch();
 }
 
@@ -601,7 +614,16 @@ size_t bsa_forward_workspace_size(int B, int H, int N, int d, int blk) {
 int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N, int d, int blk,
                 const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale, void* o,
                 float* lse, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  return bsa_forward_residual(q, k, v, B, H, N, d, blk, row_ptr, col_idx, softmax_scale, o, lse,
+                              nullptr, workspace, ws_bytes, stream);
+}
+
+int bsa_forward_residual(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                         int blk, const int32_t* row_ptr, const int32_t* col_idx,
+                         float softmax_scale, void* o, float* lse, void* o_residual,
+                         void* workspace, size_t ws_bytes, bsa_stream_t stream) {
   if (!q || !k || !v || !o || !row_ptr || !col_idx) return BSA_ERR_INVALID_ARG;
+  if (o_residual != nullptr && !aligned(o_residual, 16)) return BSA_ERR_UNSUPPORTED;
   if (workspace != nullptr && (ws_bytes < 4 || !aligned(workspace, 4))) return BSA_ERR_WORKSPACE;
   int rc = common_shape_checks(B, H, N, blk);
   if (rc != BSA_OK) return rc;
@@ -615,8 +637,10 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
   if (counter != nullptr && cudaMemsetAsync(counter, 0, sizeof(int), s) != cudaSuccess)
     return BSA_ERR_CUDA;
   if (d == 64)
-    return launch_fwd_blk<64>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);
-  return launch_fwd_blk<128>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, counter, s);
+    return launch_fwd_blk<64>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, o_residual,
+                              counter, s);
+  return launch_fwd_blk<128>(blk, q, k, v, B, H, N, row_ptr, col_idx, scale, o, lse, o_residual,
+                             counter, s);
 }
 
 size_t bsa_backward_workspace_size(int B, int H, int N, int d, int blk) {
@@ -628,8 +652,18 @@ int bsa_backward(const void* q, const void* k, const void* v, const void* o, con
                  const float* lse, int B, int H, int N, int d, int blk, const int32_t* row_ptr,
                  const int32_t* col_idx, float softmax_scale, void* dq, void* dk, void* dv,
                  void* workspace, size_t ws_bytes, bsa_stream_t stream) {
+  return bsa_backward_residual(q, k, v, o, nullptr, dout, lse, B, H, N, d, blk, row_ptr, col_idx,
+                               softmax_scale, dq, dk, dv, workspace, ws_bytes, stream);
+}
+
+int bsa_backward_residual(const void* q, const void* k, const void* v, const void* o,
+                          const void* o_residual, const void* dout, const float* lse, int B,
+                          int H, int N, int d, int blk, const int32_t* row_ptr,
+                          const int32_t* col_idx, float softmax_scale, void* dq, void* dk,
+                          void* dv, void* workspace, size_t ws_bytes, bsa_stream_t stream) {
   if (!q || !k || !v || !o || !dout || !lse || !row_ptr || !col_idx || !dq || !dk || !dv)
     return BSA_ERR_INVALID_ARG;
+  if (o_residual != nullptr && !aligned(o_residual, 16)) return BSA_ERR_UNSUPPORTED;
   int rc = common_shape_checks(B, H, N, blk);
   if (rc != BSA_OK) return rc;
   if (d != 64 && d != 128) return BSA_ERR_UNSUPPORTED;
@@ -649,14 +683,15 @@ int bsa_backward(const void* q, const void* k, const void* v, const void* o, con
   float* delta = static_cast<float*>(workspace);
   const long long tokens = (long long)B * H * N;
   const auto* ob = static_cast<const __nv_bfloat16*>(o);
+  const auto* rb = static_cast<const __nv_bfloat16*>(o_residual);
   const auto* db = static_cast<const __nv_bfloat16*>(dout);
   if (d == 64) {
-    bsa::bwd_delta_kernel<64><<<ceil_div(tokens * 8, 256), 256, 0, s>>>(ob, db, tokens, delta);
+    bsa::bwd_delta_kernel<64><<<ceil_div(tokens * 8, 256), 256, 0, s>>>(ob, rb, db, tokens, delta);
     if (check_launch()) return BSA_ERR_CUDA;
     return launch_bwd_blk<64>(blk, q, k, v, dout, B, H, N, row_ptr, col_idx, lse, delta, scale,
                               dq, dk, dv, s);
   }
-  bsa::bwd_delta_kernel<128><<<ceil_div(tokens * 16, 256), 256, 0, s>>>(ob, db, tokens, delta);
+  bsa::bwd_delta_kernel<128><<<ceil_div(tokens * 16, 256), 256, 0, s>>>(ob, rb, db, tokens, delta);
   if (check_launch()) return BSA_ERR_CUDA;
   return launch_bwd_blk<128>(blk, q, k, v, dout, B, H, N, row_ptr, col_idx, lse, delta, scale,
                              dq, dk, dv, s);
@@ -751,9 +786,10 @@ extern "C" int asa_build_mask_noalloc(const void* q, const void* k, int B, int H
     return BSA_ERR_WORKSPACE;
   void* ws = noalloc_scratch_for_current_device();
   if (ws == nullptr) return BSA_ERR_CUDA;
-  // Nothing in the scratch has to start at zero: each call's pooling kernel
-  // writes every pooled row and its selection kernel writes every bitmap word
-  // before anything reads them.
+  // The scratch keeps the previous call's contents.  What must start at zero
+  // (the selection kernel's ticket and look-back flags) is zeroed by this
+  // call's pooling kernel; everything else (pooled rows, bitmap words) is
+  // written by this call before anything reads it.
   const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
   cudaStream_t s = as_cuda(stream);
   if (d == 64)

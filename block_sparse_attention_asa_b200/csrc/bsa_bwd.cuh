@@ -111,9 +111,12 @@ struct BwdCfg {
   static constexpr uint32_t S_COL = 0, DP_COL = 128, ACC0_COL = 256, ACC1_COL = 384;
 };
 
-// D_t = dO_t . O_t, fp32; D/8 lanes per token, 16-byte loads.
+// D_t = dO_t . O_t, fp32; D/8 lanes per token, 16-byte loads.  With o_res
+// (the forward's rounding residual) O_t is taken as O_t + o_res_t, which
+// carries the forward's fp32 result.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16* __restrict__ o,
+                                                        const __nv_bfloat16* __restrict__ o_res,
                                                         const __nv_bfloat16* __restrict__ dout,
                                                         long long tokens, float* __restrict__ delta) {
   constexpr int TPT = D / 8;
@@ -130,6 +133,16 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16* __r
       const float2 fa = __bfloat1622float2(ha[e]), fb = __bfloat1622float2(hb[e]);
       acc = fmaf(fa.x, fb.x, acc);
       acc = fmaf(fa.y, fb.y, acc);
+    }
+    if (o_res != nullptr) {
+      const uint4 c = __ldg(reinterpret_cast<const uint4*>(o_res + tok * D) + part);
+      const __nv_bfloat162* hc = reinterpret_cast<const __nv_bfloat162*>(&c);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 fc = __bfloat1622float2(hc[e]), fb = __bfloat1622float2(hb[e]);
+        acc = fmaf(fc.x, fb.x, acc);
+        acc = fmaf(fc.y, fb.y, acc);
+      }
     }
   }
 #pragma unroll

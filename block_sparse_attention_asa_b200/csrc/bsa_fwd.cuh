@@ -39,23 +39,29 @@
 //               exchange their maxima through shared memory.  Raw-score max
 //               (3-input max), packed f32x2 scale/shift and sums, one ex2 per
 //               score, lazy rescale of O (only when the max grows by more than
-//               2^8; exact because the final normalisation uses the same stale
-//               max), P (bf16) written over S in TMEM.  A half whose keys all
-//               belong to blocks its q-block does not list writes P = 0 without
+//               2^kLazyRescaleLog2; exact because the final normalisation uses
+//               the same stale max), P (bf16) written over S in TMEM, or at
+//               d = 64 into its own columns.  A half whose keys all belong to
+//               blocks its q-block does not list writes P = 0 without
 //               exponentials.
 //
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D).
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D);
+// at d = 64 P_A [320,384) and P_B [448,512) (separate P), else P over S.
 //
 // Ordering facts the pipeline relies on:
 //   * tcgen05.mma ops issued by one thread execute in order, so S_X may be
 //     overwritten by the QK issued after the PV that read P_X from it;
-//   * the commit that signals S_X(t) ready also covers PV_X(t-1), issued by
-//     the same thread before QK_X(t), so the softmax may rescale O_X without a
-//     further wait;
+//   * P over S: the commit that signals S_X(t) ready also covers PV_X(t-1),
+//     issued by the same thread before QK_X(t), so the softmax may rescale O_X
+//     without a further wait.  Separate P: QK_X(t) follows the softmax's read
+//     of S_X(t-1) (s_read) and precedes PV_X(t-1); the softmax waits for
+//     PV_X(t-1) (pv_done) before it writes P_X(t) or rescales O_X;
 //   * ring index s reuses K and V slots NK and NV indices later; the PV that
 //     frees the V slot of a step is issued by its slot's thread as soon as the
-//     step's P is stored, before that thread waits for anything of its next
-//     step, so the producer never waits on work that needs its own next step;
+//     step's P is stored (separate P: right after the next QK, which needs
+//     only K tiles the producer's K front loads while its V front runs at
+//     most NV steps behind), so the producer never waits on work that needs
+//     its own next step;
 //   * the producer never stops its V front while it waits on consumer
 //     progress (a free K slot is polled; the slot's Q buffer, released by its
 //     item's last QK, is waited for with the V front running), because that
@@ -79,6 +85,7 @@ struct FwdParams {
   float scale;                    // softmax scale
   __nv_bfloat16* o;
   float* lse;
+  __nv_bfloat16* o_res;           // optional: the fp32 O minus its bf16 rounding, as bf16
   unsigned long long wait_ns;     // bound on every wait
   int* item_counter;              // zeroed before launch; null: items dealt statically
 };
@@ -100,9 +107,10 @@ struct FwdCfg {
   static constexpr int K_OFF = 2 * TILE;
   static constexpr int V_OFF = K_OFF + NK * TILE;
   static constexpr int AUX_OFF = V_OFF + NV * TILE;
-  static constexpr int BAR_BYTES = 512;
-  // k/v full+free, q/s/p/o barriers, m_full, l_full+free, drain, pair
-  static constexpr int NBARS = 2 * NK + 2 * NV + 12 + 2 * NM + 8 + 2 + 8;
+  static constexpr int BAR_BYTES = 1024;
+  // k/v full+free, q/s/p/o barriers, m_full, l_full+free, drain, pair, s_read,
+  // pv_done
+  static constexpr int NBARS = 2 * NK + 2 * NV + 12 + 2 * NM + 8 + 2 + 8 + 4;
   static_assert(NBARS * 8 <= BAR_BYTES, "mbarriers must fit their area");
   static constexpr int SMETA_OFF = AUX_OFF + BAR_BYTES;          // 2 x NM step entries
   static constexpr int SMETA_INTS = 24;
@@ -117,6 +125,9 @@ struct FwdCfg {
   static constexpr int XCH_BYTES = (2 * 2 * 2 * 128 + 2 * 2 * 128) * 4;
   static constexpr int SMEM = XCH_OFF + XCH_BYTES + 1024;
   static constexpr int S_COL = 0, O_COL = 256;
+  // d = 64: O takes 64 of its slot's 128 columns, and P (128 keys as bf16
+  // pairs) gets the other 64 instead of being written over S.
+  static constexpr bool SEP_P = D == 64;
 };
 
 // entry kinds (list headers and per-slot step entries)
@@ -136,6 +147,15 @@ constexpr int kRegControl = kSoftmaxWarps == 4 ? 80 : 72;
 constexpr int kRegSoftmax = kSoftmaxWarps == 4 ? 200 : 96;
 static_assert(128 * kRegControl + 2 * kSoftmaxWarps * 32 * kRegSoftmax <= kFwdThreads * kLaunchRegs,
               "register split over budget");
+
+// Lazy rescale: a row keeps its running max m (and the scale of O and of its
+// sum) until a step's max exceeds m by more than this many exp2 units, so P =
+// 2^((s - m) c) stays below 2^kLazyRescaleLog2.  Any value is exact (the final
+// O/l and LSE use the same m); the bound only keeps the fp32 sums finite: l
+// and O (l times a convex combination of V) stay below 2^kLazyRescaleLog2
+// times the number of keys (at most 2^23) times max|v|.  2^8 rescaled O on 14%
+// of the CogVideoX layer's steps (measured on B200); 2^20 almost never does.
+constexpr float kLazyRescaleLog2 = 20.0f;
 
 // list segment header (ints): [0] kind (0 segment, 2 end) [1] bh [2] qt [3] nq
 //                             [4] count [5] first segment [6] last segment
@@ -252,6 +272,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* l_free = l_full + 4;                 // [2][2]
   uint64_t* mma_drain = l_free + 4;             // [2]
   uint64_t* pair_bar = mma_drain + 2;            // [2 slots][4 lane quarters]
+  uint64_t* s_read = pair_bar + 8;               // [2] (separate-P mode)
+  uint64_t* pv_done = s_read + 2;                // [2] (separate-P mode)
   int* smeta = reinterpret_cast<int*>(smem + C::SMETA_OFF);
   int* hdr = reinterpret_cast<int*>(smem + C::HDR_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
@@ -288,6 +310,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     mbar_init(&mma_drain[0], 1);
     mbar_init(&mma_drain[1], 1);
     for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 2);   // one arrive per warp
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_read[x], kSoftmaxWarps);   // one arrive per softmax warp of the slot
+      mbar_init(&pv_done[x], 1);
+    }
     *abort_flag = 0;
     *mma_lock = 0;
     fence_mbar_init();
@@ -377,6 +403,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (token >= p.N) break;
             uint4* dst = reinterpret_cast<uint4*>(p.o + ((long long)st.bh * p.N + token) * D);
             for (int c = lane; c < D / 8; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
+            if (p.o_res) {
+              uint4* dr = reinterpret_cast<uint4*>(p.o_res + ((long long)st.bh * p.N + token) * D);
+              for (int c = lane; c < D / 8; c += 32) dr[c] = make_uint4(0u, 0u, 0u, 0u);
+            }
             if (lane == 0 && p.lse) p.lse[(long long)st.bh * p.N + token] = -INFINITY;
           }
           continue;
@@ -619,8 +649,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // One thread per slot: issuing a tcgen05.mma costs the issuing thread about
     // as long as the instruction runs, so a single issuer for both slots would
     // be the bottleneck.  Within a slot the order is the program order of its
-    // thread: PV_X(t-1) is issued before QK_X(t) (S_X holds P_X), and the
-    // commit that publishes S_X(t) covers PV_X(t-1).
+    // thread.  P over S: PV_X(t-1) is issued before QK_X(t) (S_X holds P_X),
+    // and the commit that publishes S_X(t) covers PV_X(t-1).  Separate P (d =
+    // 64): QK_X(t) is issued as soon as the softmax has read S_X(t-1), before
+    // PV_X(t-1), whose completion the softmax waits for (pv_done) before it
+    // writes P_X(t) or rescales O_X.
     if (lane == 0) {
       const int X = warp - 1;
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
@@ -631,6 +664,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint64_t dk0 = smem_desc(smem_u32(smem + C::K_OFF), 16, 1024);
       const uint64_t dv0 = smem_desc(smem_u32(smem + C::V_OFF), C::CHUNK, 1024);
       const uint32_t t_s = tmem + C::S_COL + X * 128, t_o = tmem + C::O_COL + X * 128;
+      const uint32_t t_p = C::SEP_P ? t_o + D : t_s;   // P: its own columns, or over S
       int pend = -1, pend_first = 0, pend_last = 0, qc = 0, pc = 0, items = 0;
       bool ok = true, issued = false;
       // A slot's group of MMAs (its PV, or its QK) runs contiguously in the
@@ -660,10 +694,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint32_t acc0 = pend_first ? 0u : 1u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(t_o, t_s + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+          mma_ts(t_o, t_p + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
                  kk == 0 ? acc0 : 1u);
         ++pc;
         mma_commit(&v_free[sp % C::NV]);
+        if (C::SEP_P) mma_commit(&pv_done[X]);
         if (pend_last) {
           mma_commit(&o_done[X]);
           ++items;
@@ -671,9 +706,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         pend = -1;
       };
       for (int t = 0; ok; ++t) {
-        // PV of the previous step as soon as its P is stored: it must precede
-        // this step's QK (S_X holds P_X) but need not wait for this step's K
-        if (pend >= 0) {
+        // P over S: PV of the previous step as soon as its P is stored; it must
+        // precede this step's QK (S_X holds P_X) but need not wait for this
+        // step's K
+        if (!C::SEP_P && pend >= 0) {
           if (!wait_pv() || !lock_mma()) { ok = false; break; }
           issue_pv();
           unlock_mma();
@@ -681,7 +717,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int mi = X * C::NM + t % C::NM;
         if (!mbar_wait(&m_full[mi], (t / C::NM) & 1, p.wait_ns)) { ok = false; break; }
         const int* sm = smeta + mi * C::SMETA_INTS;
-        if (sm[0] == kEntryEnd) break;
+        if (sm[0] == kEntryEnd) {
+          if (C::SEP_P && pend >= 0) {
+            if (!wait_pv() || !lock_mma()) { ok = false; break; }
+            issue_pv();
+            unlock_mma();
+          }
+          break;
+        }
         const int first = sm[1], lastt = sm[2], s = sm[22];
         const int ks = s % C::NK;
         if (!mbar_wait(&k_full[ks], (s / C::NK) & 1, p.wait_ns)) { ok = false; break; }
@@ -689,6 +732,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (!mbar_wait(&q_full[X], qc & 1, p.wait_ns)) { ok = false; break; }
           ++qc;
         }
+        // separate P: S_X is free once the softmax holds S_X(t-1) in registers
+        if (C::SEP_P && t > 0 && !mbar_wait(&s_read[X], (t - 1) & 1, p.wait_ns)) { ok = false; break; }
         if (!lock_mma()) { ok = false; break; }
         tc_fence_after();
         const uint64_t dk = dk0 + static_cast<uint64_t>((ks * C::TILE) >> 4);
@@ -702,6 +747,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (lastt) mma_commit(&q_free[X]);
         mma_commit(&s_full[X]);
         unlock_mma();
+        if (C::SEP_P && pend >= 0) {
+          if (!wait_pv() || !lock_mma()) { ok = false; break; }
+          issue_pv();
+          unlock_mma();
+        }
         pend = s;
         pend_first = first;
         pend_last = lastt;
@@ -749,6 +799,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     };
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t s_col = C::S_COL + X * 128, o_col = C::O_COL + X * 128;
+    const uint32_t p_col = C::SEP_P ? o_col + D : s_col;   // P: own columns or over S
+    // Separate P: P_X(t) and a rescale of O_X wait for PV_X(t-1) (pv_done),
+    // once per step, just before the first of them.
+    bool pv_pending = false;
+    auto wait_prev_pv = [&](int t) -> bool {
+      if (!C::SEP_P || !pv_pending) return true;
+      pv_pending = false;
+      const bool r = mbar_wait(&pv_done[X], (t - 1) & 1, p.wait_ns);
+      tc_fence_after();
+      return __all_sync(0xffffffffu, r);
+    };
     float* xmax = reinterpret_cast<float*>(smem + C::XCH_OFF);        // [2][2 slots][2 halves][128]
     float* xsum = xmax + 2 * 2 * 2 * 128;                             // [2 slots][2 halves][128]
     const float c2 = p.scale_log2;
@@ -807,6 +868,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
       }
       tmem_wait_ld();
+      if (C::SEP_P) {
+        // S_X(t) is in registers: the next QK may overwrite it
+        warp_arrive(&s_read[X]);
+        pv_pending = t > 0;
+      }
       float hmax = -INFINITY;
       if (!part_dead) {
         // masking: slots this row's q-block does not list, unused slots, keys >= N
@@ -846,12 +912,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       // lazy rescale (decided per warp: tcgen05.ld/st are warp-collective)
       const float m_new = fmaxf(m_run, tmax);
-      const bool grow = m_run == -INFINITY ? (m_new > -INFINITY) : ((m_new - m_run) * c2 > 8.0f);
+      const bool grow = m_run == -INFINITY ? (m_new > -INFINITY)
+                                           : ((m_new - m_run) * c2 > kLazyRescaleLog2);
       float alpha = 1.0f;
       if (grow) {
         alpha = (m_run == -INFINITY) ? 0.0f : fast_ex2((m_run - m_new) * c2);
         m_run = m_new;
       }
+      if (!wait_prev_pv(t)) { ok = false; break; }
       if (!first && __any_sync(0xffffffffu, grow)) {
         // O_X holds PV up to the previous step, complete (see header); scale
         // this warp's columns before any PV of this step
@@ -897,8 +965,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             pk[c] = *reinterpret_cast<uint32_t*>(&hb);
           }
         }
-        // P (bf16 pairs) over S: keys KW h + 32 q2 .. +31 -> columns KW/2 h + 16 q2
-        tmem_st16(t_lane + s_col + h * (KW / 2) + q2 * 16, pk);
+        // P (bf16 pairs): keys KW h + 32 q2 .. +31 -> columns KW/2 h + 16 q2
+        // (over S, or in the separate P columns)
+        tmem_st16(t_lane + p_col + h * (KW / 2) + q2 * 16, pk);
       }
       float la0, la1, lb0, lb1;
       unpack2(ls2a, la0, la1);
@@ -939,6 +1008,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int e = 0; e < 4; ++e)
               dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
                                   packed[4 * e + 3]);
+          }
+          if (p.o_res != nullptr && token < p.N) {
+            // the rounding residual of each element, so that O + residual
+            // carries the fp32 result to about 2^-16
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float a = __uint_as_float(r[2 * e]) * inv_l;
+              const float b = __uint_as_float(r[2 * e + 1]) * inv_l;
+              const float2 hi = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&packed[e]));
+              __nv_bfloat162 lo = __floats2bfloat162_rn(a - hi.x, b - hi.y);
+              packed[e] = *reinterpret_cast<uint32_t*>(&lo);
+            }
+            uint4* dr = reinterpret_cast<uint4*>(p.o_res + ((long long)e_bh * p.N + token) * D +
+                                                 h * DW + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dr[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
+                                 packed[4 * e + 3]);
           }
         }
         warp_arrive(&o_free[X]);

@@ -4,14 +4,13 @@
 // (intra-frame), M3 multi-diagonal (evenly spaced, cross-frame), M4 vertical
 // stripe (global tokens); Efficient-vDiT blog, "3.1 注意力图块化": block-wise
 // repetition of the 3D attention map (frame tiles).  The rule for each pattern
-// is stated on token pairs (see include/bsa.h); below it is evaluated per block
-// pair in closed form from the two blocks' token ranges.
+// is stated on token pairs (see include/bsa.h); below, each row's kept blocks
+// are runs of consecutive blocks in closed form from the token ranges.
 //
-// One warp per (h, q-block): lanes sweep the candidate kv-blocks, a ballot and
-// a popcount prefix give each kept block its position, and the row is written
-// once per batch index (the pattern does not depend on b).  Count pass, scan,
-// write pass.  Full and diagonal rows are contiguous ranges and skip the
-// per-block test; the output is write-bound.
+// Two kernels: one CTA per head computes the rows' counts in closed form and
+// writes row_ptr (offsets from per-pattern totals and a block scan), then one
+// warp per row writes its runs of consecutive block ids (coalesced), once per
+// batch index (the pattern does not depend on b).  The output is write-bound.
 #pragma once
 #include "common.cuh"
 
@@ -21,6 +20,7 @@ constexpr int kMaxPatternHeads = 1024;
 
 struct PatternParams {
   int B, H, N, blk, nb;
+  int lblk;                       // log2(blk): blk is a power of two
   int band_w, frame_tokens, f_lo, f_hi, stripe_blocks, tile_global_frames;
   int32_t* row_ptr;
   int32_t* col_idx;
@@ -28,112 +28,211 @@ struct PatternParams {
   int8_t head_pattern[kMaxPatternHeads];
 };
 
-// Is kv-block j kept for q-block i under `pattern`?
-__device__ __forceinline__ bool pattern_keep(const PatternParams& p, int pattern, int i, int j) {
+// ------------------------------------------------------------------ intervals
+// Every rule keeps, for q-block i, a union of a few runs of consecutive
+// kv-blocks, given in closed form by the two blocks' token ranges:
+//   diag       one run [i - w, i + w];
+//   multidiag  one run per frame offset f (the blocks whose offsets u - t can
+//              meet [fS - w blk, fS + w blk]);
+//   stripe     one run per frame t (the blocks holding tokens [tS, tS + sb blk));
+//   tile3d     the blocks sharing a frame with block i, and those holding a
+//              token of the first g frames.
+// The runs come in ascending order of their first block; touching or
+// overlapping runs are merged, so `emit(j0, j1)` sees disjoint ascending runs
+// [j0, j1] and the row's blocks are exactly their union.  With stripe_blocks
+// = 0 a frame has no stripe tokens and the stripe rule keeps nothing.
+// 32-bit arithmetic throughout: N < 2^23 (nb^2 < 2^31 per head, blk <= 128),
+// band widths are at most 2^24 tokens and frames at most 2^28 (checked on the
+// host), stripe_blocks <= nb and tile_global_frames <= the number of frames
+// (clamped on the host; neither clamp changes a mask).  The frame offsets are
+// clamped to those whose run can reach [0, nb) before any product f S.
+__device__ __forceinline__ int floor_div(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+
+// floor(a / blk): an arithmetic shift, blk being a power of two
+__device__ __forceinline__ int blk_floor(const PatternParams& p, int a) { return a >> p.lblk; }
+
+// Smallest kv-block j whose last token is >= a (nb when none).
+__device__ __forceinline__ int first_block_ending_at_or_after(const PatternParams& p, int a) {
+  int j = blk_floor(p, a);   // (j+1) blk - 1 >= a  <=>  j >= floor(a / blk)
+  if (j < 0) j = 0;
+  if (j >= p.nb - 1) return (p.N - 1 >= a) ? p.nb - 1 : p.nb;
+  return j;
+}
+
+template <typename Emit>
+__device__ __forceinline__ void pattern_runs(const PatternParams& p, int pattern, int i,
+                                             Emit&& emit) {
+  const int nb = p.nb, blk = p.blk, S = p.frame_tokens;
+  int ps = -1, pe = -2;   // pending run
+  auto add = [&](int j0, int j1) {
+    if (j0 < 0) j0 = 0;
+    if (j1 > nb - 1) j1 = nb - 1;
+    if (j0 > j1) return;
+    if (ps >= 0 && j0 <= pe + 1) {
+      if (j1 > pe) pe = j1;
+      return;
+    }
+    if (ps >= 0) emit(ps, pe);
+    ps = j0;
+    pe = j1;
+  };
+  const int ti_lo = i * blk, ti_hi = min(p.N, ti_lo + blk) - 1;
   switch (pattern) {
     case BSA_PATTERN_FULL:
-      return true;
+      add(0, nb - 1);
+      break;
     case BSA_PATTERN_SKIP:
-      return false;
+      break;
     case BSA_PATTERN_DIAG:
-      return abs(i - j) <= p.band_w;
+      add(i - p.band_w, i + p.band_w);
+      break;
+    case BSA_PATTERN_MULTIDIAG: {
+      // offsets u - t over the two blocks form [uj_lo - ti_hi, uj_hi - ti_lo];
+      // it meets [c - wb, c + wb] (c = f S) iff uj_lo <= c + wb + ti_hi and
+      // uj_hi >= c - wb + ti_lo; only the f whose run can reach [0, nb) matter
+      const int wb = p.band_w * blk;
+      int f0 = p.f_lo, f1 = p.f_hi;
+      const int fa = -floor_div(wb + ti_hi, S);                 // ceil((-wb - ti_hi) / S)
+      const int fb = floor_div(p.N - 1 + wb - ti_lo, S);
+      if (f0 < fa) f0 = fa;
+      if (f1 > fb) f1 = fb;
+      for (int f = f0; f <= f1; ++f) {
+        const int c = f * S;
+        add(first_block_ending_at_or_after(p, c - wb + ti_lo), blk_floor(p, c + wb + ti_hi));
+      }
+      break;
+    }
+    case BSA_PATTERN_STRIPE: {
+      const int L = p.stripe_blocks * blk;
+      if (L <= 0) break;
+      if (L >= S) {   // every token of every frame is a stripe token
+        add(0, nb - 1);
+        break;
+      }
+      for (int t0 = 0; t0 < p.N; t0 += S) add(blk_floor(p, t0), blk_floor(p, min(p.N, t0 + L) - 1));
+      break;
+    }
+    case BSA_PATTERN_TILE3D: {
+      if (p.tile_global_frames > 0)   // blocks holding a token of the first g frames
+        add(0, blk_floor(p, min(p.N, p.tile_global_frames * S) - 1));
+      const int fi_lo = ti_lo / S, fi_hi = ti_hi / S;
+      add(first_block_ending_at_or_after(p, fi_lo * S), blk_floor(p, min(p.N, (fi_hi + 1) * S) - 1));
+      break;
+    }
     default:
       break;
   }
-  // token ranges of the two blocks (N < 2^31, so 32-bit arithmetic is exact)
-  const int blk = p.blk, S = p.frame_tokens;
-  const int ti_lo = i * blk, ti_hi = min(p.N, ti_lo + blk) - 1;
-  const int uj_lo = j * blk, uj_hi = min(p.N, uj_lo + blk) - 1;
-  if (pattern == BSA_PATTERN_MULTIDIAG) {
-    // offsets u - t over the two blocks: [lo, hi]; frame offset f is hit when
-    // [lo, hi] meets [f*S - w*blk, f*S + w*blk] (a few f: no division)
-    const long long lo = (long long)uj_lo - ti_hi, hi = (long long)uj_hi - ti_lo;
-    const long long wb = (long long)p.band_w * blk;
-    if (p.f_hi - p.f_lo <= 8) {
-      for (int f = p.f_lo; f <= p.f_hi; ++f) {
-        const long long c = (long long)f * S;
-        if (lo <= c + wb && hi >= c - wb) return true;
-      }
-      return false;
+  if (ps >= 0) emit(ps, pe);
+}
+
+__device__ __forceinline__ int pattern_count(const PatternParams& p, int pattern, int i) {
+  int n = 0;
+  pattern_runs(p, pattern, i, [&](int j0, int j1) { n += j1 - j0 + 1; });
+  return n;
+}
+
+constexpr int kPatternScanThreads = 1024;
+constexpr int kPatternIds = BSA_PATTERN_TILE3D + 1;
+
+// One CTA per head h: the row counts in closed form, their prefix within the
+// head, and the head's offset from the totals of the patterns of the heads
+// before it (each pattern's total is computed once) -> row_ptr of every row
+// (b, h, i), for all b.  No scratch memory is needed.  A total past INT32_MAX
+// is recorded as BSA_ERR_CAPACITY.
+__global__ void __launch_bounds__(kPatternScanThreads) pattern_rowptr_kernel(
+    const __grid_constant__ PatternParams p) {
+  __shared__ long long s_tot[kPatternIds];
+  __shared__ long long s_warp[kPatternScanThreads / 32];
+  __shared__ long long s_carry;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int h = blockIdx.x;
+  if (tid < kPatternIds) s_tot[tid] = 0;
+  __syncthreads();
+  // totals of the patterns in use
+  bool used[kPatternIds] = {};
+  for (int hh = 0; hh < p.H; ++hh) used[p.head_pattern[hh]] = true;
+  for (int pid = 0; pid < kPatternIds; ++pid) {
+    if (!used[pid]) continue;
+    long long part = 0;
+    for (int i = tid; i < p.nb; i += kPatternScanThreads) part += pattern_count(p, pid, i);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) atomicAdd(reinterpret_cast<unsigned long long*>(&s_tot[pid]),
+                             static_cast<unsigned long long>(part));
+  }
+  __syncthreads();
+  long long base = 0, total = 0;
+  for (int hh = 0; hh < p.H; ++hh) {
+    const long long t = s_tot[p.head_pattern[hh]];
+    if (hh < h) base += t;
+    total += t;
+  }
+  if ((long long)p.B * total > 0x7fffffffLL) {
+    if (tid == 0) record_error(BSA_ERR_CAPACITY);
+    return;
+  }
+  // prefix over the head's rows, kPatternScanThreads rows at a time
+  const int pid = p.head_pattern[h];
+  if (tid == 0) s_carry = 0;
+  __syncthreads();
+  for (int i0 = 0; i0 < p.nb; i0 += kPatternScanThreads) {
+    const int i = i0 + tid;
+    const long long c = i < p.nb ? pattern_count(p, pid, i) : 0;
+    long long incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
     }
-    // many offsets: the f range that [lo, hi] can reach, in closed form
-    const long long a = lo - wb, bb = hi + wb;
-    long long fmin = a >= 0 ? (a + S - 1) / S : -((-a) / S);    // ceil(a / S)
-    long long fmax = bb >= 0 ? bb / S : -((-bb + S - 1) / S);   // floor(bb / S)
-    fmin = max(fmin, (long long)p.f_lo);
-    fmax = min(fmax, (long long)p.f_hi);
-    return fmin <= fmax;
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+      const long long w = s_warp[lane];
+      long long wi = w;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long v = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += v;
+      }
+      s_warp[lane] = wi - w;
+    }
+    __syncthreads();
+    const long long carry = s_carry;
+    const long long end = carry + s_warp[warp] + incl;   // inclusive, within the head
+    if (i < p.nb)
+      for (int b = 0; b < p.B; ++b)
+        p.row_ptr[((long long)b * p.H + h) * p.nb + i + 1] =
+            static_cast<int32_t>((long long)b * total + base + end);
+    __syncthreads();
+    if (tid == kPatternScanThreads - 1) s_carry = end;
+    __syncthreads();
   }
-  if (pattern == BSA_PATTERN_STRIPE) {
-    const int f = uj_lo / S;
-    return (long long)(uj_lo - f * S) < (long long)p.stripe_blocks * blk ||
-           (long long)(f + 1) * S <= uj_hi;
-  }
-  if (pattern == BSA_PATTERN_TILE3D) {
-    const int fi_lo = ti_lo / S, fi_hi = ti_hi / S, fj_lo = uj_lo / S, fj_hi = uj_hi / S;
-    return (fj_lo <= fi_hi && fj_hi >= fi_lo) || fj_lo < p.tile_global_frames;
-  }
-  return false;
+  if (h == 0 && tid == 0) p.row_ptr[0] = 0;
 }
 
-__device__ __forceinline__ void pattern_range(const PatternParams& p, int pattern, int i, int& j0,
-                                              int& j1) {
-  j0 = 0;
-  j1 = p.nb;
-  if (pattern == BSA_PATTERN_SKIP) {
-    j1 = 0;
-  } else if (pattern == BSA_PATTERN_DIAG) {
-    j0 = max(0, i - p.band_w);
-    j1 = min(p.nb, i + p.band_w + 1);
-  }
-}
-
-// kWrite = false: store the row's count at row_ptr[r+1] for every b.
-// kWrite = true : write col_idx[row_ptr[r] ...] for every b.
-template <bool kWrite>
-__global__ void __launch_bounds__(256) pattern_kernel(const __grid_constant__ PatternParams p) {
+// One warp per row (h, i), every b: the runs, written as consecutive block
+// ids from the row's start (coalesced); nothing past the capacity is written.
+__global__ void __launch_bounds__(256) pattern_write_kernel(const __grid_constant__ PatternParams p) {
   const int lane = threadIdx.x & 31;
   const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (unit >= (long long)p.H * p.nb) return;
   const int h = static_cast<int>(unit / p.nb), i = static_cast<int>(unit % p.nb);
   const int pattern = p.head_pattern[h];
-  int j0, j1;
-  pattern_range(p, pattern, i, j0, j1);
-  if (!kWrite) {
-    int cnt = 0;
-    if (pattern == BSA_PATTERN_FULL || pattern == BSA_PATTERN_SKIP || pattern == BSA_PATTERN_DIAG) {
-      cnt = j1 - j0;
-    } else {
-      for (int j = j0 + lane; j < j1; j += 32) cnt += pattern_keep(p, pattern, i, j) ? 1 : 0;
-      cnt = warp_sum(cnt);
-    }
-    if (lane == 0)
-      for (int b = 0; b < p.B; ++b) p.row_ptr[((long long)b * p.H + h) * p.nb + i + 1] = cnt;
-    return;
-  }
-  // Full and diagonal rows are one contiguous range: no per-block test.  The
-  // row's bounds are read once per batch index, outside the block sweep.
-  const bool contiguous = pattern == BSA_PATTERN_FULL || pattern == BSA_PATTERN_DIAG;
-  const unsigned lt = (1u << lane) - 1u;
   for (int b = 0; b < p.B; ++b) {
     const long long r = ((long long)b * p.H + h) * p.nb + i;
-    const long long base = p.row_ptr[r], end = p.row_ptr[r + 1];
-    int pos = 0;
-    for (int jb = j0; jb < j1; jb += 32) {
-      const int j = jb + lane;
-      const bool keep = j < j1 && (contiguous || pattern_keep(p, pattern, i, j));
-      const unsigned m = __ballot_sync(0xffffffffu, keep);
-      if (keep) {
-        const long long at = base + pos + __popc(m & lt);
-        if (at < end) {
-          if (at < p.capacity)
-            p.col_idx[at] = j;
-          else
-            record_error(BSA_ERR_CAPACITY);
-        }
+    const long long start = p.row_ptr[r], end = p.row_ptr[r + 1];
+    long long pos = start;
+    pattern_runs(p, pattern, i, [&](int j0, int j1) {
+      const int n = j1 - j0 + 1;
+      for (int k = lane; k < n; k += 32) {
+        const long long at = pos + k;
+        if (at < end && at < p.capacity)
+          p.col_idx[at] = static_cast<int32_t>(j0 + k);
+        else if (at >= p.capacity && lane == 0)
+          record_error(BSA_ERR_CAPACITY);
       }
-      pos += __popc(m);
-    }
+      pos += n;
+    });
   }
 }
 

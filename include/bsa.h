@@ -94,6 +94,8 @@ typedef struct CUstream_st* bsa_stream_t; /* same object as cudaStream_t */
  *   5. union with the diagonal block i (keep_diag != 0) and blocks
  *      [0, n_sink_blocks);
  *   6. write CSR (row_ptr, col_idx ascending).
+ * Two kernels: pooling (reads q and k once), then scores, selection and the
+ * CSR write together (the row offsets by a decoupled look-back across CTAs).
  * Selection runs in fp32 on the device: rows whose result depends on scores
  * within fp32 rounding of the cut may differ from an exact evaluation.
  * q, k: bf16 [B,H,N,d].  col_capacity: entries available in col_idx; if the mask
@@ -123,8 +125,10 @@ int asa_build_mask(const void* q, const void* k, int B, int H, int N, int d, int
  * calls no cudaMalloc, cudaFree or other allocating routine.
  * The first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture begins.  Every call on a device shares the one array, and
- * the array keeps the last call's contents (nothing in it needs to start at
+ * any stream capture begins.  The address is kept for the life of the
+ * process: do not reset the device (cudaDeviceReset) between calls.  Every
+ * call on a device shares the one array, and the array keeps the last call's
+ * contents (each call clears, on the device, the part that must start at
  * zero): calls that may overlap on the GPU -- on different streams, or from
  * different host threads without ordering -- race on it and must be
  * serialized by the caller. */
@@ -150,7 +154,8 @@ int asa_build_mask_noalloc(const void* q, const void* k, int B, int H, int N, in
  * synchronizes `stream` once after counting, stores the mask's nnz there, and
  * returns BSA_ERR_CAPACITY (writing no col_idx) when col_capacity < nnz.  With
  * nnz_out_host NULL the call is fully asynchronous and an overflow is reported
- * through the device status.  No workspace. */
+ * through the device status.  No workspace.  band_w*blk above 2^24 or
+ * frame_tokens above 2^28 gives BSA_ERR_UNSUPPORTED. */
 int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
                  int band_w, int frame_tokens, int f_lo, int f_hi, int stripe_blocks,
                  int tile_global_frames, int32_t* row_ptr, int32_t* col_idx,
@@ -178,6 +183,18 @@ int bsa_forward(const void* q, const void* k, const void* v, int B, int H, int N
                 float softmax_scale, void* o, float* lse,
                 void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
+/* bsa_forward that also writes, when o_residual is not NULL (bf16
+ * [B,H,N,d], 16-byte aligned, caller-owned), each element's fp32 result minus
+ * its bf16 rounding in o, rounded to bf16: o + o_residual carries the fp32 O
+ * to about 2^-16 relative.  bsa_backward_residual takes it to form D = dO.O
+ * from the fp32 O (an empty row gives o_residual = 0).  The pages have no
+ * counterpart; it is the training path's precision option (see
+ * bsa_backward_residual).  Misaligned o_residual: BSA_ERR_UNSUPPORTED. */
+int bsa_forward_residual(const void* q, const void* k, const void* v, int B, int H, int N, int d,
+                         int blk, const int32_t* row_ptr, const int32_t* col_idx,
+                         float softmax_scale, void* o, float* lse, void* o_residual,
+                         void* workspace, size_t ws_bytes, bsa_stream_t stream);
+
 /* ---- gradients of attention over kept blocks --------------------------------
  * [BLADE] 技术框架: ASA is trained jointly with the step distillation, so the
  * attention over the kept blocks is differentiated.  For a given dO (bf16
@@ -204,6 +221,18 @@ int bsa_backward(const void* q, const void* k, const void* v, const void* o, con
                  const int32_t* row_ptr, const int32_t* col_idx, float softmax_scale,
                  void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                  bsa_stream_t stream);
+
+/* bsa_backward with the forward's rounding residual (bsa_forward_residual;
+ * NULL: the same as bsa_backward).  With it D_t = dO_t.(o_t + o_residual_t)
+ * comes from the fp32 O; without it D comes from the bf16 o, whose rounding
+ * (up to 2^-8 relative per element) then reaches dq through D -- on peaked
+ * attention, where dP - D nearly cancels, that rounding dominates dq's error.
+ * dk and dv are barely affected.  Misaligned o_residual: BSA_ERR_UNSUPPORTED. */
+int bsa_backward_residual(const void* q, const void* k, const void* v, const void* o,
+                          const void* o_residual, const void* dout, const float* lse, int B,
+                          int H, int N, int d, int blk, const int32_t* row_ptr,
+                          const int32_t* col_idx, float softmax_scale, void* dq, void* dk,
+                          void* dv, void* workspace, size_t ws_bytes, bsa_stream_t stream);
 
 /* ---- Sparse-vDiT offline pattern search (diagnostic) ------------------------
  * Sparse-vDiT blog, "核心公式 / 离线搜索损失函数", "注意力模式选择" and

@@ -30,8 +30,11 @@ def test_status_strings(lib):
 
 
 def test_workspace_and_capacity_sizes(lib):
-    # Wan2.1-shaped layer: q̄,k̄ fp32 (2*6144*128*4) + bitmaps (6144*16*4)
-    assert bsa.asa_workspace_size(1, 12, 32760, 128, 64) == 2 * 6144 * 128 * 4 + 6144 * 16 * 4
+    # Wan2.1-shaped layer: q̄,k̄ fp32 (2*6144*128*4) + bitmaps (6144*16*4) + the
+    # select kernels' look-back state (a 256-byte ticket area, one 8-byte flag
+    # per row)
+    assert bsa.asa_workspace_size(1, 12, 32760, 128, 64) == (2 * 6144 * 128 * 4 + 6144 * 16 * 4 +
+                                                             256 + 6144 * 8)
     assert bsa.asa_max_nnz(1, 12, 32760, 64, bsa.MODE_MASS, 0, 0.1, 0, 0) == 6144 * 51
     assert bsa.asa_max_nnz(2, 48, 17776, 64, bsa.MODE_TOPK, 33, 0.0, 0, 4) == 2 * 48 * 278 * 37
     assert bsa.asa_max_nnz(1, 2, 128, 16, bsa.MODE_TOPK, 3, 0.0, 1, 0) == 16 * 4

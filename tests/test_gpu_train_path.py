@@ -2,7 +2,11 @@
 and the backward on the bench's full layers.
 
 * block_sparse_attention (one autograd node over bsa_forward / bsa_backward)
-  returns exactly the kernels' O and gradients;
+  returns exactly the kernels' O and gradients (the residual path);
+* with the forward's rounding residual, D comes from the fp32 O and dQ meets
+  the plain gradient bounds, with no term for O's bf16 rounding, on the
+  PE-structured tiny layer where that term dominated; the residual is at most
+  half an ulp of o;
 * on the Wan and Cog layers (GPU mask -> forward -> backward), 16 random
   q-blocks plus the last (dQ) and 16 random kv-blocks plus the first and last
   (dK, dV) match the oracle's per-block restatement
@@ -33,8 +37,8 @@ def test_autograd_node_returns_the_kernels_gradients(cuda_lib):
     qa, ka, va = (t.clone().requires_grad_(True) for t in (q, k, v))
     o = cuda_lib.block_sparse_attention(qa, ka, va, blk, rpd, cid)
     o.backward(do)
-    o2, lse = cuda_lib.bsa_forward(q, k, v, blk, rpd, cid)
-    dq, dk, dv = cuda_lib.bsa_backward(q, k, v, o2, do, lse, blk, rpd, cid)
+    o2, lse, res = cuda_lib.bsa_forward(q, k, v, blk, rpd, cid, residual=True)
+    dq, dk, dv = cuda_lib.bsa_backward(q, k, v, o2, do, lse, blk, rpd, cid, o_residual=res)
     assert cuda_lib.check_device_status() == 0
     assert torch.equal(o.detach(), o2)
     for got, want in ((qa.grad, dq), (ka.grad, dk), (va.grad, dv)):
@@ -114,3 +118,30 @@ def test_tiny_sequences_end_to_end(cuda_lib, N, d, blk):
     probs = oracle.attention_probs(qf, kf, blk, rp_h, ci_h)
     zb = zero_gradient_bounds(qf, kf, vf, dof, oh, o_ref, probs, 1.0 / np.sqrt(d))
     compare_gradients([x.float().cpu().numpy() for x in (dq, dk, dv)], ref, term, zb)
+
+
+@pytest.mark.parametrize("w", [W.TINY, W.COG], ids=lambda w: w.name)
+def test_residual_backward_meets_plain_bounds(cuda_lib, w):
+    # bsa_forward_residual / bsa_backward_residual: dQ within rel-RMS 1e-2 and
+    # max 2e-2 of max|ref| with no allowance for O's rounding (R20); on the
+    # Cog layer a few sampled heads keep the oracle fast
+    q, k, v = W.make_qkv(w)
+    if w is W.COG:
+        q, k, v = (t[:1, :2].contiguous() for t in (q, k, v))
+    B, H, N, d = q.shape
+    g = torch.Generator().manual_seed(1234)
+    do = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    qd, kd, vd, dod = (t.cuda() for t in (q, k, v, do))
+    rp, ci = cuda_lib.asa_build_mask(qd, kd, w.blk, w.mode, w.topk, w.mass_tau, w.max_keep_ratio,
+                                     w.keep_diag, w.n_sink_blocks)
+    o, lse, res = cuda_lib.bsa_forward(qd, kd, vd, w.blk, rp, ci, residual=True)
+    dq, dk, dv = cuda_lib.bsa_backward(qd, kd, vd, o, dod, lse, w.blk, rp, ci, o_residual=res)
+    assert cuda_lib.check_device_status() == 0
+    # the residual is at most half an ulp of o (2^-8 |o|), up to its own bf16
+    # rounding
+    assert torch.all(res.float().abs() <= o.float().abs() * (2.0 ** -8) * (1 + 2.0 ** -7))
+    rp_h, ci_h = rp.cpu().numpy().astype(np.int64), ci.cpu().numpy()
+    qf, kf, vf, dof = W.as_f64(q), W.as_f64(k), W.as_f64(v), W.as_f64(do)
+    ref = oracle.attention_backward(qf, kf, vf, dof, w.blk, rp_h, ci_h)
+    rel = compare_gradients([x.float().cpu().numpy() for x in (dq, dk, dv)], ref, None)
+    assert rel[0][0] <= 1e-2
