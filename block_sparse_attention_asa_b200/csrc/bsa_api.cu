@@ -121,8 +121,10 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   if (!make_map(&mq, q, B * H, N, D, 128) || !make_map(&mk, k, B * H, N, D, BLK) ||
       !make_map(&mv, v, B * H, N, D, BLK))
     return BSA_ERR_CUDA;
-  static DeviceFlags smem_set;
-  if (!allow_smem(bsa::bsa_fwd_kernel<D, BLK>, C::SMEM, smem_set)) return BSA_ERR_CUDA;
+  static DeviceFlags smem_set, smem_set_res;
+  if (!allow_smem(bsa::bsa_fwd_kernel<D, BLK, false>, C::SMEM, smem_set) ||
+      !allow_smem(bsa::bsa_fwd_kernel<D, BLK, true>, C::SMEM, smem_set_res))
+    return BSA_ERR_CUDA;
   bsa::FwdParams p;
   p.B = B;
   p.H = H;
@@ -144,7 +146,10 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   if (sms <= 0) return BSA_ERR_CUDA;
   // persistent: one CTA per SM, two item slots per CTA
   const int grid = std::min(sms, ceil_div(p.n_items, 2));
-  bsa::bsa_fwd_kernel<D, BLK><<<grid, bsa::kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, p);
+  if (o_res != nullptr)
+    bsa::bsa_fwd_kernel<D, BLK, true><<<grid, bsa::kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, p);
+  else
+    bsa::bsa_fwd_kernel<D, BLK, false><<<grid, bsa::kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, p);
   return check_launch();
 }
 

@@ -248,7 +248,9 @@ struct SchedSlot {
   bool done = false;
 };
 
-template <int D, int BLK>
+// RES: also write O's rounding residual (p.o_res); a separate instantiation so
+// that the plain forward carries none of its code.
+template <int D, int BLK, bool RES>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -403,7 +405,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             if (token >= p.N) break;
             uint4* dst = reinterpret_cast<uint4*>(p.o + ((long long)st.bh * p.N + token) * D);
             for (int c = lane; c < D / 8; c += 32) dst[c] = make_uint4(0u, 0u, 0u, 0u);
-            if (p.o_res) {
+            if (RES) {
               uint4* dr = reinterpret_cast<uint4*>(p.o_res + ((long long)st.bh * p.N + token) * D);
               for (int c = lane; c < D / 8; c += 32) dr[c] = make_uint4(0u, 0u, 0u, 0u);
             }
@@ -1009,7 +1011,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
                                   packed[4 * e + 3]);
           }
-          if (p.o_res != nullptr && token < p.N) {
+          if (RES && token < p.N) {
             // the rounding residual of each element, so that O + residual
             // carries the fp32 result to about 2^-16
 #pragma unroll
