@@ -37,8 +37,9 @@ brute-force subset enumeration; patterns vs token-pair enumeration; the
 invariants of a convex combination; a hand-computable worked example; the
 gradients vs torch float64 autograd of SDPA and vs central finite differences
 of the forward oracle, with the softmax's shift and scaling identities.  The
-3D-tile pattern's block reading has only its own token-level definition to
-check against: its parity beyond that is unpinned.
+3D-tile pattern is pinned by a hand derivation for frames that straddle
+blocks (``tests/golden/tile3d_example.json``); the block reading it checks is
+the plainest one the Efficient-vDiT page's section 3.1 allows.
 """
 from .asa import pool, pooled_probs, select_row, asa_mask, MaskInfo  # noqa: F401
 from .patterns import pattern_row, pattern_mask, keep_token_pair  # noqa: F401
