@@ -144,8 +144,8 @@ int launch_fwd(const void* q, const void* k, const void* v, int B, int H, int N,
   p.item_counter = item_counter;
   const int sms = sm_count();
   if (sms <= 0) return BSA_ERR_CUDA;
-  // persistent: one CTA per SM, two item slots per CTA
-  const int grid = std::min(sms, ceil_div(p.n_items, 2));
+  // persistent: one CTA per SM, one stream of items per CTA
+  const int grid = std::min(sms, p.n_items);
   if (o_res != nullptr)
     bsa::bsa_fwd_kernel<D, BLK, true><<<grid, bsa::kFwdThreads, C::SMEM, stream>>>(mq, mk, mv, p);
   else

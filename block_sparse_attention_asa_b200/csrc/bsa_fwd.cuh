@@ -11,64 +11,62 @@
 // an M=64 or N=64 tcgen05.mma runs at half the rate of M=N=128, so a 128x128
 // step with some masked work beats exact 64-row tiles.
 //
-// Persistent CTAs (one per SM), each running TWO independent item slots (A, B)
-// so that one slot's softmax overlaps the other slot's MMAs.  Slot X of CTA c
-// starts on item 2c+X; every later item comes from a grid-wide counter, so the
-// SMs that run faster take more items (without a counter, items 2c+X+2kG of a
-// static deal, G = grid size).
+// Persistent CTAs (one per SM), each running ONE stream of steps over its
+// items, with the score tile S double-buffered in TMEM so that the tensor pipe
+// runs the next step's QK (and the previous step's PV) while the softmax works
+// on the current step, and with O and Q double-buffered per item so that the
+// stream does not stop at item boundaries.  CTA c starts on item c; every later
+// item comes from a grid-wide counter, so the SMs that run faster take more
+// items (without a counter, items c + kG of a static deal, G = grid size).
 //
-// Warp roles (640 threads, 20 warps):
+// Warp roles (384 threads, 12 warps):
 //   warp 3      scheduler: per item builds the q-block bitmaps of its CSR rows
 //               and the ascending union list (block id + keep bits) in shared
-//               memory, in segments, double-buffered per slot, and prefetches
-//               the item's Q tile into L2.
+//               memory, in segments, double-buffered, and prefetches the
+//               item's Q tile into L2.
 //   warp 0      producer (one lane, state in registers): per step takes up to
-//               128/blk list entries, publishes a per-slot step entry (ring
-//               index, first/last, block ids, keep bits) and the gathered K
-//               boxes (TMA, 128B swizzle) into a K ring, alternating slots; the
-//               V boxes follow on a separate front, since V is needed one step
-//               later than K.
-//   warps 1, 2  MMA issuers, one thread per slot: S_X = Q_X Kᵀ, then for the
-//               previous step O_X += P_X V with P read from TMEM.  Issuing a
-//               tcgen05.mma costs the issuing thread about as long as the MMA
-//               runs (measured on B200), so each slot has its own issuer.
-//   warp 2      also allocates and releases TMEM.
-//   warps 4-11  softmax + epilogue of slot A;  warps 12-19 the same for slot B.
-//               Warp (q, h): rows 32q..32q+31 (TMEM lane quarter q), keys
-//               64h..64h+63 of each 128-key step; the two halves of a row
-//               exchange their maxima through shared memory.  Raw-score max
-//               (3-input max), packed f32x2 scale/shift and sums, one ex2 per
-//               score, lazy rescale of O (only when the max grows by more than
-//               2^kLazyRescaleLog2; exact because the final normalisation uses
-//               the same stale max), P (bf16) written over S in TMEM, or at
-//               d = 64 into its own columns.  A half whose keys all belong to
-//               blocks its q-block does not list writes P = 0 without
-//               exponentials.
+//               128/blk list entries, publishes a step entry (first/last, block
+//               ids, keep bits) and the gathered K boxes (TMA, 128B swizzle)
+//               into a K ring; the V boxes follow on a separate front, since V
+//               is needed one step later than K.  Q tiles go into two buffers,
+//               by item parity.
+//   warp 1      MMA issuer (one thread): S(t) = Q Kᵀ into S buffer t%2, then
+//               O += P(t-1) V for the previous step, with P read from TMEM.
+//   warp 2      allocates and releases TMEM.
+//   warps 4-11  softmax + epilogue.  Warp (q, h): rows 32q..32q+31 (TMEM lane
+//               quarter q), keys 64h..64h+63 of each 128-key step; the two
+//               halves of a row exchange their maxima through shared memory.
+//               Raw-score max (3-input max), packed f32x2 scale/shift and sums,
+//               one ex2 per score, lazy rescale of O (only when the max grows
+//               by more than 2^kLazyRescaleLog2; exact because the final
+//               normalisation uses the same stale max), P (bf16) written over
+//               S in TMEM.  A half whose keys all belong to blocks its q-block
+//               does not list writes P = 0 without exponentials.  An item's
+//               epilogue (O / l to bf16, LSE) runs after the next item's first
+//               step, by which time its last PV has long finished.
 //
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+D), O_B [384,384+D);
-// at d = 64 P_A [320,384) and P_B [448,512) (separate P), else P over S.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
 //
-// Ordering facts the pipeline relies on:
-//   * tcgen05.mma ops issued by one thread execute in order, so S_X may be
-//     overwritten by the QK issued after the PV that read P_X from it;
-//   * P over S: the commit that signals S_X(t) ready also covers PV_X(t-1),
-//     issued by the same thread before QK_X(t), so the softmax may rescale O_X
-//     without a further wait.  Separate P: QK_X(t) follows the softmax's read
-//     of S_X(t-1) (s_read) and precedes PV_X(t-1); the softmax waits for
-//     PV_X(t-1) (pv_done) before it writes P_X(t) or rescales O_X;
+// Issue order of the single MMA thread: QK(0), QK(1), PV(0), QK(2), PV(1), ...
+// i.e. in step t's slot: QK(t) into S(t%2), then PV(t-1).  Ordering facts:
+//   * tcgen05.mma ops issued by one thread execute in order.  QK(t) overwrites
+//     S(t%2) after PV(t-2) read P(t-2) from it (PV(t-2) was issued first, and
+//     waited for the softmax to finish step t-2);
+//   * when the softmax sees S(t) ready, QK(t), and so PV(t-2), have completed:
+//     only PV(t-1) may still run.  A rescale of O at step t (same item) waits
+//     for PV(t-1) (pv_done, one phase per PV, so the wait is unambiguous);
+//   * per-buffer barriers (S ready, P stored, O done/free, Q full/free) are
+//     indexed by step or item parity; each phase is waited for before the
+//     buffer can be reused, so every parity wait is unambiguous;
 //   * ring index s reuses K and V slots NK and NV indices later; the PV that
-//     frees the V slot of a step is issued by its slot's thread as soon as the
-//     step's P is stored (separate P: right after the next QK, which needs
-//     only K tiles the producer's K front loads while its V front runs at
-//     most NV steps behind), so the producer never waits on work that needs
-//     its own next step;
+//     frees the V slot of a step is issued as soon as the step's P is stored,
+//     and needs no K tile the producer has not loaded, so the producer never
+//     waits on work that needs its own next step;
 //   * the producer never stops its V front while it waits on consumer
-//     progress (a free K slot is polled; the slot's Q buffer, released by its
-//     item's last QK, is waited for with the V front running), because that
-//     progress may itself need a V tile only this thread's V front loads;
-//   * a barrier phase is never completed twice before its waiter looks: each
-//     "free" barrier is released only after the front that waits on it has
-//     passed the entry, so every parity wait is unambiguous;
+//     progress (a free K slot is polled; the Q buffer, released by the last QK
+//     of the item two before, is waited for with the V front running),
+//     because that progress may itself need a V tile only this thread's V
+//     front loads;
 //   * every wait is bounded (BSA_ERR_TIMEOUT on expiry, then the CTA unwinds).
 #pragma once
 #include "common.cuh"
@@ -90,63 +88,10 @@ struct FwdParams {
   int* item_counter;              // zeroed before launch; null: items dealt statically
 };
 
-template <int D, int BLK>
-struct FwdCfg {
-  static constexpr int SLOTS = 128 / BLK;            // kv-blocks per step
-  static constexpr int QB = 128 / BLK;               // q-blocks per tile
-  static constexpr int NCH = D / 64;                 // 64-column swizzle chunks
-  static constexpr int TILE = 128 * D * 2;           // bytes of a 128-row tile
-  static constexpr int CHUNK = 128 * 128;            // bytes of one 128x64 chunk
-  static constexpr int NK = D == 128 ? 2 : 4;        // K ring depth
-  static constexpr int NV = D == 128 ? 2 : 4;        // V ring depth
-  static constexpr int NM = 8;                       // per-slot softmax entries
-  static constexpr int LCAP = 512;                   // union entries per list segment
-  static constexpr int RW = LCAP / 32;               // bitmap words per fill round (<= LCAP bits)
-  static_assert(RW >= 1 && RW <= 32, "fill round must fit one warp and one segment");
-  static constexpr int Q_OFF = 0;                    // Q_A, Q_B
-  static constexpr int K_OFF = 2 * TILE;
-  static constexpr int V_OFF = K_OFF + NK * TILE;
-  static constexpr int AUX_OFF = V_OFF + NV * TILE;
-  static constexpr int BAR_BYTES = 1024;
-  // k/v full+free, q/s/p/o barriers, m_full, l_full+free, drain, pair, s_read,
-  // pv_done
-  static constexpr int NBARS = 2 * NK + 2 * NV + 12 + 2 * NM + 8 + 2 + 8 + 4;
-  static_assert(NBARS * 8 <= BAR_BYTES, "mbarriers must fit their area");
-  static constexpr int SMETA_OFF = AUX_OFF + BAR_BYTES;          // 2 x NM step entries
-  static constexpr int SMETA_INTS = 24;
-  static constexpr int VQ = 8;                                   // V-front queue entries
-  static constexpr int VQ_INTS = VQ * 12;                        // producer V-front queue
-  static constexpr int HDR_OFF = SMETA_OFF + (2 * NM * SMETA_INTS + VQ_INTS) * 4;  // 2x2 headers x 8 ints
-  static constexpr int MISC_OFF = HDR_OFF + 2 * 2 * 8 * 4;
-  static constexpr int LIST_OFF = MISC_OFF + 64;                 // 2 slots x 2 bufs x LCAP
-  static constexpr int BM_OFF = LIST_OFF + 2 * 2 * LCAP * 4;     // per-slot bitmaps
-  static constexpr int kMaxBitmapBytes = 4096;                   // per slot
-  static constexpr int XCH_OFF = BM_OFF + 2 * kMaxBitmapBytes;   // row max / sum exchange
-  static constexpr int XCH_BYTES = (2 * 2 * 2 * 128 + 2 * 2 * 128) * 4;
-  static constexpr int SMEM = XCH_OFF + XCH_BYTES + 1024;
-  static constexpr int S_COL = 0, O_COL = 256;
-  // d = 64: O takes 64 of its slot's 128 columns, and P (128 keys as bf16
-  // pairs) gets the other 64 instead of being written over S.
-  static constexpr bool SEP_P = D == 64;
-};
-
-// entry kinds (list headers and per-slot step entries)
-constexpr int kEntryNormal = 0, kEntryEnd = 2;
-
-// Softmax warps per slot: 4 (one per TMEM lane quarter, a thread owns all 128
-// keys of its row) or 8 (two per lane quarter, 64 keys each, the two halves
-// exchanging their row maxima).
+// Softmax warps: two per TMEM lane quarter, 64 keys each, the two halves
+// exchanging their row maxima.
 constexpr int kSoftmaxWarps = 8;
-constexpr int kFwdThreads = (4 + 2 * kSoftmaxWarps) * 32;
-// Register split (setmaxnreg, per warpgroup): the control warpgroup (producer,
-// MMA issuers, scheduler) gives registers to the softmax warpgroups.  The sum
-// must not exceed the launch allocation (threads x the per-thread launch
-// limit), or the increase would wait forever.
-constexpr int kLaunchRegs = kSoftmaxWarps == 4 ? 168 : 96;
-constexpr int kRegControl = kSoftmaxWarps == 4 ? 80 : 72;
-constexpr int kRegSoftmax = kSoftmaxWarps == 4 ? 200 : 96;
-static_assert(128 * kRegControl + 2 * kSoftmaxWarps * 32 * kRegSoftmax <= kFwdThreads * kLaunchRegs,
-              "register split over budget");
+constexpr int kFwdThreads = (4 + kSoftmaxWarps) * 32;
 
 // Lazy rescale: a row keeps its running max m (and the scale of O and of its
 // sum) until a step's max exceeds m by more than this many exp2 units, so P =
@@ -157,11 +102,53 @@ static_assert(128 * kRegControl + 2 * kSoftmaxWarps * 32 * kRegSoftmax <= kFwdTh
 // of the CogVideoX layer's steps (measured on B200); 2^20 almost never does.
 constexpr float kLazyRescaleLog2 = 20.0f;
 
+template <int D, int BLK>
+struct FwdCfg {
+  static constexpr int SLOTS = 128 / BLK;            // kv-blocks per step
+  static constexpr int QB = 128 / BLK;               // q-blocks per tile
+  static constexpr int NCH = D / 64;                 // 64-column swizzle chunks
+  static constexpr int TILE = 128 * D * 2;           // bytes of a 128-row tile
+  static constexpr int CHUNK = 128 * 128;            // bytes of one 128x64 chunk
+  static constexpr int NK = D == 128 ? 2 : 4;        // K ring depth
+  static constexpr int NV = D == 128 ? 2 : 4;        // V ring depth
+  static constexpr int NM = 8;                       // step entries
+  static constexpr int LCAP = 512;                   // union entries per list segment
+  static constexpr int RW = LCAP / 32;               // bitmap words per fill round (<= LCAP bits)
+  static_assert(RW >= 1 && RW <= 32, "fill round must fit one warp and one segment");
+  static_assert(NM > NK + 2, "a step entry is reused only after its step's P is stored");
+  static constexpr int Q_OFF = 0;                    // Q0, Q1 (item parity)
+  static constexpr int K_OFF = 2 * TILE;
+  static constexpr int V_OFF = K_OFF + NK * TILE;
+  static constexpr int AUX_OFF = V_OFF + NV * TILE;
+  static constexpr int BAR_BYTES = 512;
+  // k/v full+free, q full/free, s_full, p_full, o done/free, m_full, l
+  // full/free, drain, pair, pv_done
+  static constexpr int NBARS = 2 * NK + 2 * NV + 2 * 6 + NM + 4 + 1 + 4 + 1;
+  static_assert(NBARS * 8 <= BAR_BYTES, "mbarriers must fit their area");
+  static constexpr int SMETA_OFF = AUX_OFF + BAR_BYTES;          // NM step entries
+  static constexpr int SMETA_INTS = 24;
+  static constexpr int VQ = 8;                                   // V-front queue entries
+  static constexpr int VQ_INTS = VQ * 12;                        // producer V-front queue
+  static constexpr int HDR_OFF = SMETA_OFF + (NM * SMETA_INTS + VQ_INTS) * 4;   // 2 headers x 8 ints
+  static constexpr int MISC_OFF = HDR_OFF + 2 * 8 * 4;
+  static constexpr int LIST_OFF = MISC_OFF + 64;                 // 2 bufs x LCAP
+  static constexpr int BM_OFF = LIST_OFF + 2 * LCAP * 4;         // q-block bitmaps
+  static constexpr int kMaxBitmapBytes = 4096;
+  static constexpr int XCH_OFF = BM_OFF + kMaxBitmapBytes;       // row max / sum exchange
+  static constexpr int XCH_BYTES = (2 * 2 * 128 + 2 * 128) * 4;
+  static constexpr int SMEM = XCH_OFF + XCH_BYTES + 1024;
+  static_assert(SMEM <= 227 * 1024, "shared memory over the per-CTA limit");
+  static constexpr int S_COL = 0, O_COL = 256;
+};
+
+// entry kinds (list headers and step entries)
+constexpr int kEntryNormal = 0, kEntryEnd = 2;
+
 // list segment header (ints): [0] kind (0 segment, 2 end) [1] bh [2] qt [3] nq
 //                             [4] count [5] first segment [6] last segment
 // list entry: kv-block id | (keep bits over the tile's q-blocks) << 16
 
-// per-slot softmax entry, as ints:
+// step entry, as ints:
 //  [0] kind (0 normal, 2 end)  [1] first  [2] last  [3] nvalid  [4] bh  [5] qt
 //  [6..13] block ids          [14..21] keep bits (q-blocks of the tile)
 //  [22] ring index of the step (K slot = ring % NK, V slot = ring % NV)
@@ -226,18 +213,17 @@ __device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* m, int c0,
                : "memory");
 }
 
-// Producer state of one item slot (kept in registers: always named, never indexed).
+// Producer state (kept in registers).
 struct ProdSlot {
   int sc = 0;         // list segments consumed so far
   int pos = 0, count = 0;
   int bh = 0, qt = 0, nq = 0;
-  int tcount = 0;     // softmax entries published
   int qcount = 0;     // Q tiles loaded
   bool have = false, lastseg = false, first_tile = false, flushed = false;
   bool need_q = false;  // the current item's Q tile is not loaded yet
 };
 
-// Scheduler state of one item slot.
+// Scheduler state.
 struct SchedSlot {
   int item = 0;       // current item
   int fills = 0;      // segments published
@@ -263,26 +249,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* k_free = k_full + C::NK;             // [NK]
   uint64_t* v_full = k_free + C::NK;             // [NV]
   uint64_t* v_free = v_full + C::NV;             // [NV]
-  uint64_t* q_full = v_free + C::NV;             // [2]
+  uint64_t* q_full = v_free + C::NV;             // [2] by item parity
   uint64_t* q_free = q_full + 2;                 // [2]
-  uint64_t* s_full = q_free + 2;                 // [2]
-  uint64_t* p_full = s_full + 2;                 // [2]
-  uint64_t* o_done = p_full + 2;                 // [2]
+  uint64_t* s_full = q_free + 2;                 // [2] by step parity
+  uint64_t* p_full = s_full + 2;                 // [2] by step parity
+  uint64_t* o_done = p_full + 2;                 // [2] by item parity
   uint64_t* o_free = o_done + 2;                 // [2]
-  uint64_t* m_full = o_free + 2;                 // [2][NM]
-  uint64_t* l_full = m_full + 2 * C::NM;         // [2][2]
-  uint64_t* l_free = l_full + 4;                 // [2][2]
-  uint64_t* mma_drain = l_free + 4;             // [2]
-  uint64_t* pair_bar = mma_drain + 2;            // [2 slots][4 lane quarters]
-  uint64_t* s_read = pair_bar + 8;               // [2] (separate-P mode)
-  uint64_t* pv_done = s_read + 2;                // [2] (separate-P mode)
+  uint64_t* m_full = o_free + 2;                 // [NM]
+  uint64_t* l_full = m_full + C::NM;             // [2]
+  uint64_t* l_free = l_full + 2;                 // [2]
+  uint64_t* mma_drain = l_free + 2;              // [1]
+  uint64_t* pair_bar = mma_drain + 1;            // [4 lane quarters]
+  uint64_t* pv_done = pair_bar + 4;              // [1] one phase per PV
   int* smeta = reinterpret_cast<int*>(smem + C::SMETA_OFF);
   int* hdr = reinterpret_cast<int*>(smem + C::HDR_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   int* abort_flag = reinterpret_cast<int*>(smem + C::MISC_OFF + 4);
-  int* mma_lock = reinterpret_cast<int*>(smem + C::MISC_OFF + 8);   // 0 free, X+1 held by slot X
   uint32_t* lists = reinterpret_cast<uint32_t*>(smem + C::LIST_OFF);
-  uint32_t* bm_all = reinterpret_cast<uint32_t*>(smem + C::BM_OFF);
+  uint32_t* bm = reinterpret_cast<uint32_t*>(smem + C::BM_OFF);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nbw = p.nbw;
@@ -300,24 +284,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&q_full[x], 1);
       mbar_init(&q_free[x], 1);
       mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], kSoftmaxWarps);   // one arrive per softmax warp of the slot
+      mbar_init(&p_full[x], kSoftmaxWarps);   // one arrive per softmax warp
       mbar_init(&o_done[x], 1);
       mbar_init(&o_free[x], kSoftmaxWarps);
-      for (int s = 0; s < C::NM; ++s) mbar_init(&m_full[x * C::NM + s], 1);
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&l_full[x * 2 + b], 1);
-        mbar_init(&l_free[x * 2 + b], 1);
-      }
+      mbar_init(&l_full[x], 1);
+      mbar_init(&l_free[x], 1);
     }
-    mbar_init(&mma_drain[0], 1);
-    mbar_init(&mma_drain[1], 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&pair_bar[i], 2);   // one arrive per warp
-    for (int x = 0; x < 2; ++x) {
-      mbar_init(&s_read[x], kSoftmaxWarps);   // one arrive per softmax warp of the slot
-      mbar_init(&pv_done[x], 1);
-    }
+    for (int s = 0; s < C::NM; ++s) mbar_init(&m_full[s], 1);
+    mbar_init(mma_drain, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 2);   // one arrive per warp
+    mbar_init(pv_done, 1);
     *abort_flag = 0;
-    *mma_lock = 0;
     fence_mbar_init();
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
@@ -333,39 +310,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 3) {
-    regs_dec<kRegControl>();
     // ================================================================ scheduler
-    // Per slot: next item, its q-block bitmaps, then the ascending union list
-    // in segments of at most LCAP entries.  Each slot starts on item 2c + X;
-    // later items come from a grid-wide counter, so SMs that run faster take
-    // more items (without a counter: round-robin, 2c + X + 2kG).
-    SchedSlot S0, S1;
-    S0.item = 2 * blockIdx.x;
-    S1.item = 2 * blockIdx.x + 1;
+    // Next item, its q-block bitmaps, then the ascending union list in
+    // segments of at most LCAP entries.  CTA c starts on item c; later items
+    // come from a grid-wide counter, so SMs that run faster take more items
+    // (without a counter: round-robin, c + kG).
+    SchedSlot st;
+    st.item = blockIdx.x;
     auto next_item = [&](int cur) -> int {
-      if (p.item_counter == nullptr) return cur + 2 * static_cast<int>(gridDim.x);
+      if (p.item_counter == nullptr) return cur + static_cast<int>(gridDim.x);
       int v = 0;
-      if (lane == 0) v = 2 * static_cast<int>(gridDim.x) + atomicAdd(p.item_counter, 1);
+      if (lane == 0) v = static_cast<int>(gridDim.x) + atomicAdd(p.item_counter, 1);
       return __shfl_sync(0xffffffffu, v, 0);
     };
     uint64_t t_last = global_ns();
-    auto publish = [&](SchedSlot& st, int X) -> bool {
+    auto publish = [&]() -> bool {
       // returns true if a segment (or the end marker) was published
       const int b = st.fills & 1;
       if (st.fills >= 2) {
         // one lane polls, the warp follows its answer
-        bool ready = lane == 0 && mbar_try_wait(&l_free[X * 2 + b], ((st.fills >> 1) - 1) & 1);
+        bool ready = lane == 0 && mbar_try_wait(&l_free[b], ((st.fills >> 1) - 1) & 1);
         if (!__shfl_sync(0xffffffffu, ready, 0)) return false;
       }
-      int* h = hdr + (X * 2 + b) * 8;
-      uint32_t* list = lists + (X * 2 + b) * C::LCAP;
-      uint32_t* bm = bm_all + X * (C::kMaxBitmapBytes / 4);
+      int* h = hdr + b * 8;
+      uint32_t* list = lists + b * C::LCAP;
       bool first_seg = false;
       while (!st.mid) {
         if (st.item >= p.n_items) {
           if (lane == 0) {
             h[0] = kEntryEnd;
-            mbar_arrive(&l_full[X * 2 + b]);
+            mbar_arrive(&l_full[b]);
           }
           __syncwarp();
           st.done = true;
@@ -457,19 +431,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         h[4] = n;
         h[5] = first_seg;
         h[6] = last_seg;
-        mbar_arrive(&l_full[X * 2 + b]);
+        mbar_arrive(&l_full[b]);
       }
       __syncwarp();
       st.mid = !last_seg;
       ++st.fills;
       return true;
     };
-    while (!(S0.done && S1.done)) {
+    while (!st.done) {
       if (__any_sync(0xffffffffu, *(volatile int*)abort_flag != 0)) break;
-      bool prog = false;
-      if (!S0.done) prog |= publish(S0, 0);
-      if (!S1.done) prog |= publish(S1, 1);
-      if (prog) {
+      if (publish()) {
         t_last = global_ns();
       } else if (global_ns() - t_last > p.wait_ns) {
         if (lane == 0) record_error(BSA_ERR_TIMEOUT);
@@ -478,19 +449,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
     }
   } else if (warp == 0) {
-    regs_dec<kRegControl>();
     // ================================================================ producer
-    // Two fronts over the ring: the K front publishes entry sk (ring and
-    // softmax entries, K boxes) once K slot sk % NK is free; the V front loads
-    // the V boxes of entry sv < sk once V slot sv % NV is free.  V is needed one
-    // entry later than K, so a PV still running never holds back the next K.
+    // Two fronts over the ring: the K front publishes entry sk (step entry, K
+    // boxes) once K slot sk % NK is free; the V front loads the V boxes of
+    // entry sv < sk once V slot sv % NV is free.  V is needed one entry later
+    // than K, so a PV still running never holds back the next K.
     if (lane == 0) {
-      ProdSlot P0, P1;
+      ProdSlot P;
       int sk = 0, sv = 0;  // next ring index for K / for V
-      int last = 1;        // slot of the previous ring entry
-      bool ok = true, k_done = false;
-      int* vq = smeta + 2 * C::NM * C::SMETA_INTS;   // V-front queue: 8 entries x 12 ints
-      // One K-front entry for slot X.  Returns false on a wait that gave up.
+      bool ok = true;
+      int* vq = smeta + C::NM * C::SMETA_INTS;   // V-front queue: VQ entries x 12 ints
       bool used_ring = false;
       // One pass of the V front: loads every V tile whose slot is free.
       auto v_front = [&]() -> bool {
@@ -510,23 +478,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         return moved;
       };
-      auto k_step = [&](ProdSlot& P, int X) -> bool {
+      // One K-front entry.  Returns false on a wait that gave up.
+      auto k_step = [&]() -> bool {
         used_ring = false;
         int* vqe = vq + (sk % C::VQ) * 12;
         if (!P.have || P.pos == P.count) {
           if (P.have) {
-            mbar_arrive(&l_free[X * 2 + ((P.sc - 1) & 1)]);
+            mbar_arrive(&l_free[(P.sc - 1) & 1]);
             P.have = false;
           }
           const int b = P.sc & 1;
-          if (!mbar_wait(&l_full[X * 2 + b], (P.sc >> 1) & 1, p.wait_ns)) return false;
-          const int* h = hdr + (X * 2 + b) * 8;
+          if (!mbar_wait(&l_full[b], (P.sc >> 1) & 1, p.wait_ns)) return false;
+          const int* h = hdr + b * 8;
           ++P.sc;
           if (h[0] == kEntryEnd) {
-            // slot finished: END entry for its softmax and MMA threads (no ring slot)
-            int* sm = smeta + (X * C::NM + P.tcount % C::NM) * C::SMETA_INTS;
+            // stream finished: END entry for the softmax and MMA threads (no ring slot)
+            int* sm = smeta + (sk % C::NM) * C::SMETA_INTS;
             sm[0] = kEntryEnd;
-            mbar_arrive(&m_full[X * C::NM + P.tcount % C::NM]);
+            mbar_arrive(&m_full[sk % C::NM]);
             P.flushed = true;
             return true;
           }
@@ -544,26 +513,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
         }
         if (P.need_q) {
-          // Q tile, after the previous item's last QK on this slot.  While
-          // waiting, keep the V front going: that QK follows a PV whose V tile
-          // this same thread's V front may still have to load.
-          if (P.qcount > 0 && !mbar_try_wait(&q_free[X], (P.qcount - 1) & 1)) {
+          // Q tile into buffer qcount % 2, after the last QK of the item two
+          // before.  While waiting, keep the V front going: that QK follows a
+          // PV whose V tile this same thread's V front may still have to load.
+          const int qb = P.qcount & 1;
+          if (P.qcount >= 2 && !mbar_try_wait(&q_free[qb], ((P.qcount >> 1) - 1) & 1)) {
             const uint64_t t0 = global_ns();
-            while (!mbar_try_wait(&q_free[X], (P.qcount - 1) & 1)) {
+            while (!mbar_try_wait(&q_free[qb], ((P.qcount >> 1) - 1) & 1)) {
               v_front();
               if (global_ns() - t0 > p.wait_ns) return false;
             }
           }
-          mbar_arrive_expect_tx(&q_full[X], C::TILE);
+          mbar_arrive_expect_tx(&q_full[qb], C::TILE);
 #pragma unroll
           for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(smem + C::Q_OFF + X * C::TILE + c * C::CHUNK, &tm_q, &q_full[X], c * 64,
+            tma_load_3d(smem + C::Q_OFF + qb * C::TILE + c * C::CHUNK, &tm_q, &q_full[qb], c * 64,
                         P.qt * 128, P.bh);
           ++P.qcount;
           P.need_q = false;
         }
-        const uint32_t* list = lists + (X * 2 + ((P.sc - 1) & 1)) * C::LCAP;
-        int* sm = smeta + (X * C::NM + P.tcount % C::NM) * C::SMETA_INTS;
+        const uint32_t* list = lists + ((P.sc - 1) & 1) * C::LCAP;
+        int* sm = smeta + (sk % C::NM) * C::SMETA_INTS;
         const int nvalid = min(C::SLOTS, P.count - P.pos);
         const uint32_t e0 = list[P.pos];
 #pragma unroll
@@ -587,9 +557,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         sm[4] = P.bh;
         sm[5] = P.qt;
         sm[22] = sk;   // ring index: K slot sk % NK, V slot sk % NV
-        mbar_arrive(&m_full[X * C::NM + P.tcount % C::NM]);
+        mbar_arrive(&m_full[sk % C::NM]);
         used_ring = true;
-        ++P.tcount;
         const int ks = sk % C::NK;
         mbar_arrive_expect_tx(&k_full[ks], C::TILE);
 #pragma unroll
@@ -606,25 +575,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         bool prog = false;
         // ---- K front
         // (the K front stays less than VQ entries ahead of the V front, whose
-        // queue entry it writes)
-        if (!k_done && sk - sv < C::VQ &&
+        // queue entry it writes; entry sk reuses the step entry of sk - NM,
+        // whose step's P was stored before QK(sk - NK) was issued)
+        if (!P.flushed && sk - sv < C::VQ &&
             (sk < C::NK || mbar_try_wait(&k_free[sk % C::NK], ((sk / C::NK) - 1) & 1))) {
-          int X = last ^ 1;
-          const bool f0 = P0.flushed, f1 = P1.flushed;
-          if ((X == 0 && f0) || (X == 1 && f1)) X ^= 1;
-          if (f0 && f1) {
-            k_done = true;
-          } else {
-            ok = (X == 0) ? k_step(P0, 0) : k_step(P1, 1);
-            if (!ok) break;
-            last = X;
-            if (used_ring) ++sk;
-          }
+          ok = k_step();
+          if (!ok) break;
+          if (used_ring) ++sk;
           prog = true;
         }
         // ---- V front
         if (v_front()) prog = true;
-        if (k_done && sv == sk) break;
+        if (P.flushed && sv == sk) break;
         if (prog) {
           t_last = global_ns();
         } else if (global_ns() - t_last > p.wait_ns) {
@@ -641,103 +603,71 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_wait(&k_full[t % C::NK], (t / C::NK) & 1, p.wait_ns);
       for (int t = sv > C::NV ? sv - C::NV : 0; t < sv; ++t)
         mbar_wait(&v_full[t % C::NV], (t / C::NV) & 1, p.wait_ns);
-      if (P0.qcount > 0) mbar_wait(&q_full[0], (P0.qcount - 1) & 1, p.wait_ns);
-      if (P1.qcount > 0) mbar_wait(&q_full[1], (P1.qcount - 1) & 1, p.wait_ns);
+      for (int t = P.qcount > 2 ? P.qcount - 2 : 0; t < P.qcount; ++t)
+        mbar_wait(&q_full[t & 1], (t >> 1) & 1, p.wait_ns);
     }
     __syncwarp();
-  } else if (warp == 1 || warp == 2) {
-    regs_dec<kRegControl>();
-    // ================================================================ MMA issuers
-    // One thread per slot: issuing a tcgen05.mma costs the issuing thread about
-    // as long as the instruction runs, so a single issuer for both slots would
-    // be the bottleneck.  Within a slot the order is the program order of its
-    // thread.  P over S: PV_X(t-1) is issued before QK_X(t) (S_X holds P_X),
-    // and the commit that publishes S_X(t) covers PV_X(t-1).  Separate P (d =
-    // 64): QK_X(t) is issued as soon as the softmax has read S_X(t-1), before
-    // PV_X(t-1), whose completion the softmax waits for (pv_done) before it
-    // writes P_X(t) or rescales O_X.
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    // One thread issues every MMA of the CTA, in the order QK(t), PV(t-1):
+    // QK(t) needs only K(t) (and, on an item's first step, its Q tile), so the
+    // tensor pipe computes S(t) while the softmax works on step t-1; PV(t-1)
+    // waits until that step's P is stored.
     if (lane == 0) {
-      const int X = warp - 1;
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       // descriptor bases; per-instruction offsets are compile-time adds to the
       // address field (addresses stay below 2^18, so the 14-bit field never carries)
-      const uint64_t dq = smem_desc(smem_u32(smem + C::Q_OFF + X * C::TILE), 16, 1024);
+      const uint64_t dq0 = smem_desc(smem_u32(smem + C::Q_OFF), 16, 1024);
       const uint64_t dk0 = smem_desc(smem_u32(smem + C::K_OFF), 16, 1024);
       const uint64_t dv0 = smem_desc(smem_u32(smem + C::V_OFF), C::CHUNK, 1024);
-      const uint32_t t_s = tmem + C::S_COL + X * 128, t_o = tmem + C::O_COL + X * 128;
-      const uint32_t t_p = C::SEP_P ? t_o + D : t_s;   // P: its own columns, or over S
-      int pend = -1, pend_first = 0, pend_last = 0, qc = 0, pc = 0, items = 0;
+      int pend = -1, pend_first = 0, pend_last = 0, pend_item = 0;
+      int items = 0, cur_item = -1;
       bool ok = true, issued = false;
-      // A slot's group of MMAs (its PV, or its QK) runs contiguously in the
-      // tensor pipe: the other slot's issuer waits while a group is being
-      // issued.  Interleaved at instruction level, both slots' S would land
-      // late together; grouped, one lands early and the slots drift apart.
-      auto lock_mma = [&]() -> bool {
-        const uint64_t t0 = global_ns();
-        while (atomicCAS(mma_lock, 0, X + 1) != 0) {
-          if (*(volatile int*)abort_flag) return false;
-          if (global_ns() - t0 > p.wait_ns) return false;
-        }
-        return true;
-      };
-      auto unlock_mma = [&]() { atomicExch(mma_lock, 0); };
-      auto wait_pv = [&]() -> bool {
+      auto issue_pv = [&]() -> bool {
         const int sp = pend;
+        const int ob = pend_item & 1;
         if (!mbar_wait(&v_full[sp % C::NV], (sp / C::NV) & 1, p.wait_ns)) return false;
-        if (pend_first && items > 0 && !mbar_wait(&o_free[X], (items - 1) & 1, p.wait_ns))
+        // the first PV of an item overwrites its O buffer: the epilogue of
+        // the item two before must have read it
+        if (pend_first && pend_item >= 2 &&
+            !mbar_wait(&o_free[ob], ((pend_item >> 1) - 1) & 1, p.wait_ns))
           return false;
-        return mbar_wait(&p_full[X], pc & 1, p.wait_ns);
-      };
-      auto issue_pv = [&]() {
-        const int sp = pend;
+        if (!mbar_wait(&p_full[sp & 1], (sp >> 1) & 1, p.wait_ns)) return false;
         tc_fence_after();
+        const uint32_t t_o = tmem + C::O_COL + ob * 128;
+        const uint32_t t_p = tmem + C::S_COL + (sp & 1) * 128;   // P over S
         const uint64_t dv = dv0 + static_cast<uint64_t>(((sp % C::NV) * C::TILE) >> 4);
         const uint32_t acc0 = pend_first ? 0u : 1u;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           mma_ts(t_o, t_p + kk * 8, dv + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
                  kk == 0 ? acc0 : 1u);
-        ++pc;
         mma_commit(&v_free[sp % C::NV]);
-        if (C::SEP_P) mma_commit(&pv_done[X]);
-        if (pend_last) {
-          mma_commit(&o_done[X]);
-          ++items;
-        }
+        mma_commit(pv_done);
+        if (pend_last) mma_commit(&o_done[ob]);
         pend = -1;
+        return true;
       };
       for (int t = 0; ok; ++t) {
-        // P over S: PV of the previous step as soon as its P is stored; it must
-        // precede this step's QK (S_X holds P_X) but need not wait for this
-        // step's K
-        if (!C::SEP_P && pend >= 0) {
-          if (!wait_pv() || !lock_mma()) { ok = false; break; }
-          issue_pv();
-          unlock_mma();
-        }
-        const int mi = X * C::NM + t % C::NM;
+        const int mi = t % C::NM;
         if (!mbar_wait(&m_full[mi], (t / C::NM) & 1, p.wait_ns)) { ok = false; break; }
         const int* sm = smeta + mi * C::SMETA_INTS;
         if (sm[0] == kEntryEnd) {
-          if (C::SEP_P && pend >= 0) {
-            if (!wait_pv() || !lock_mma()) { ok = false; break; }
-            issue_pv();
-            unlock_mma();
-          }
+          if (pend >= 0 && !issue_pv()) ok = false;
           break;
         }
         const int first = sm[1], lastt = sm[2], s = sm[22];
         const int ks = s % C::NK;
         if (!mbar_wait(&k_full[ks], (s / C::NK) & 1, p.wait_ns)) { ok = false; break; }
         if (first) {
-          if (!mbar_wait(&q_full[X], qc & 1, p.wait_ns)) { ok = false; break; }
-          ++qc;
+          cur_item = items++;
+          if (!mbar_wait(&q_full[cur_item & 1], (cur_item >> 1) & 1, p.wait_ns)) { ok = false; break; }
         }
-        // separate P: S_X is free once the softmax holds S_X(t-1) in registers
-        if (C::SEP_P && t > 0 && !mbar_wait(&s_read[X], (t - 1) & 1, p.wait_ns)) { ok = false; break; }
-        if (!lock_mma()) { ok = false; break; }
         tc_fence_after();
+        // S(t % 2) was last read as P(t-2) by PV(t-2), issued before this QK
+        const uint32_t t_s = tmem + C::S_COL + (t & 1) * 128;
+        const uint64_t dq = dq0 + static_cast<uint64_t>(((cur_item & 1) * C::TILE) >> 4);
         const uint64_t dk = dk0 + static_cast<uint64_t>((ks * C::TILE) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -746,44 +676,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         issued = true;
         mma_commit(&k_free[ks]);
-        if (lastt) mma_commit(&q_free[X]);
-        mma_commit(&s_full[X]);
-        unlock_mma();
-        if (C::SEP_P && pend >= 0) {
-          if (!wait_pv() || !lock_mma()) { ok = false; break; }
-          issue_pv();
-          unlock_mma();
-        }
+        if (lastt) mma_commit(&q_free[cur_item & 1]);
+        mma_commit(&s_full[t & 1]);
+        if (pend >= 0 && !issue_pv()) { ok = false; break; }
         pend = s;
         pend_first = first;
         pend_last = lastt;
+        pend_item = cur_item;
       }
       if (!ok) {
         record_error(BSA_ERR_TIMEOUT);
         *(volatile int*)abort_flag = 1;
       }
       if (issued) {
-        mma_commit(&mma_drain[X]);
-        mbar_wait(&mma_drain[X], 0, p.wait_ns);
+        mma_commit(mma_drain);
+        mbar_wait(mma_drain, 0, p.wait_ns);
       }
     }
     __syncwarp();
   } else if (warp >= 4) {
-    regs_inc<kRegSoftmax>();
     // ================================================================ softmax
-    // kSoftmaxWarps warps per slot (slot A first).  Warp (q, h): q = TMEM lane
-    // quarter (rows 32q..32q+31), h = key part (keys KW*h .. KW*h+KW-1 of each
-    // 128-key step, NH parts).  With two parts, the halves of a row agree on
-    // the running max through shared memory and a two-warp mbarrier.
+    // Warp (q, h): q = TMEM lane quarter (rows 32q..32q+31), h = key part
+    // (keys KW*h .. KW*h+KW-1 of each 128-key step).  The two halves of a row
+    // agree on the running max through shared memory and a two-warp mbarrier.
     constexpr int NH = kSoftmaxWarps / 4;     // key parts per row
     constexpr int KW = 128 / NH;              // keys per warp and step
     constexpr int DW = D / NH;                // O columns per warp in rescale and epilogue
-    const int X = (warp - 4) / kSoftmaxWarps;
-    const int h = ((warp - 4) >> 2) % NH;
+    static_assert(NH == 2, "the max exchange pairs two warps");
+    const int h = (warp - 4) >> 2;
     const int wq = warp & 3;                  // TMEM lane quarter
     const int row = wq * 32 + lane;           // query row in the tile
     const int qq = row / BLK;                 // its q-block in the tile
-    uint64_t* pbar = &pair_bar[X * 4 + wq];   // the two warps of this lane quarter (NH = 2)
+    uint64_t* pbar = &pair_bar[wq];           // the two warps of this lane quarter
     int puse = 0;
     // every lane's prior shared-memory writes and tcgen05 operations are
     // ordered before lane 0's arrive by the warp barrier
@@ -800,35 +724,85 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       return __all_sync(0xffffffffu, r);
     };
     const uint32_t t_lane = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t s_col = C::S_COL + X * 128, o_col = C::O_COL + X * 128;
-    const uint32_t p_col = C::SEP_P ? o_col + D : s_col;   // P: own columns or over S
-    // Separate P: P_X(t) and a rescale of O_X wait for PV_X(t-1) (pv_done),
-    // once per step, just before the first of them.
-    bool pv_pending = false;
-    auto wait_prev_pv = [&](int t) -> bool {
-      if (!C::SEP_P || !pv_pending) return true;
-      pv_pending = false;
-      const bool r = mbar_wait(&pv_done[X], (t - 1) & 1, p.wait_ns);
-      tc_fence_after();
-      return __all_sync(0xffffffffu, r);
-    };
-    float* xmax = reinterpret_cast<float*>(smem + C::XCH_OFF);        // [2][2 slots][2 halves][128]
-    float* xsum = xmax + 2 * 2 * 2 * 128;                             // [2 slots][2 halves][128]
+    float* xmax = reinterpret_cast<float*>(smem + C::XCH_OFF);        // [2 step parity][2 halves][128]
+    float* xsum = xmax + 2 * 2 * 128;                                 // [2 halves][128]
     const float c2 = p.scale_log2;
     float m_run = -INFINITY;   // running max of raw scores (same in every part of a row)
     float l_run = 0.f;         // this part's running sum
-    int items = 0;
+    int items = 0, cur_item = -1;
     bool ok = true;
+    // an item's epilogue, deferred until the next item's first step is done
+    bool pe = false;
+    int pe_item = 0, pe_bh = 0, pe_qt = 0;
+    float pe_m = 0.f, pe_l = 0.f;
+    auto epilogue = [&]() -> bool {
+      const int ob = pe_item & 1;
+      const uint32_t o_col = C::O_COL + ob * 128;
+      const int token = pe_qt * 128 + row;
+      bool w_ok = mbar_wait(&o_done[ob], (pe_item >> 1) & 1, p.wait_ns);
+      if (!__all_sync(0xffffffffu, w_ok)) return false;
+      tc_fence_after();
+      float* xs = xsum;
+      xs[h * 128 + row] = pe_l;
+      if (!pair_sync()) return false;
+      const float l_tot = pe_l + xs[(h ^ 1) * 128 + row];
+      const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
+      __nv_bfloat16* orow = p.o + ((long long)pe_bh * p.N + token) * D + h * DW;
+#pragma unroll 1
+      for (int c = 0; c < DW / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(t_lane + o_col + h * DW + c * 32, r);
+        tmem_wait_ld();
+        uint32_t packed[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * inv_l,
+                                                    __uint_as_float(r[2 * e + 1]) * inv_l);
+          packed[e] = *reinterpret_cast<uint32_t*>(&hb);
+        }
+        if (token < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
+                                packed[4 * e + 3]);
+        }
+        if (RES && token < p.N) {
+          // the rounding residual of each element, so that O + residual
+          // carries the fp32 result to about 2^-16
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = __uint_as_float(r[2 * e]) * inv_l;
+            const float b = __uint_as_float(r[2 * e + 1]) * inv_l;
+            const float2 hi = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&packed[e]));
+            __nv_bfloat162 lo = __floats2bfloat162_rn(a - hi.x, b - hi.y);
+            packed[e] = *reinterpret_cast<uint32_t*>(&lo);
+          }
+          uint4* dr = reinterpret_cast<uint4*>(p.o_res + ((long long)pe_bh * p.N + token) * D +
+                                               h * DW + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dr[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
+                               packed[4 * e + 3]);
+        }
+      }
+      warp_arrive(&o_free[ob]);
+      if (h == 0 && p.lse != nullptr && token < p.N)
+        p.lse[(long long)pe_bh * p.N + token] =
+            l_tot > 0.f ? (pe_m * p.scale + logf(l_tot)) : -INFINITY;
+      pe = false;
+      return true;
+    };
     // kv-block slots overlapping this warp's keys
     constexpr int SPW = BLK <= KW ? KW / BLK : 1;
     const int sl0 = BLK <= KW ? h * SPW : 0;
     const uint32_t warp_mask = ((1u << SPW) - 1u) << sl0;
     for (int t = 0;; ++t) {
-      const int mi = X * C::NM + t % C::NM;
+      const int mi = t % C::NM;
       bool w_ok = mbar_wait(&m_full[mi], (t / C::NM) & 1, p.wait_ns) && !*(volatile int*)abort_flag;
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       // the entry stays valid until this step's P is published; bh/qt are kept
-      // in registers for the epilogue, which runs after that
+      // in registers for the epilogue, which runs later
       const int* sm = smeta + mi * C::SMETA_INTS;
       if (sm[0] == kEntryEnd) break;
       const int first = sm[1], lastt = sm[2], nvalid = sm[3];
@@ -851,10 +825,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const bool live_all = (live_bits & warp_mask) == warp_mask &&
                             (part_slot < sl0 || part_slot >= sl0 + SPW);
       if (first) {
+        cur_item = items++;
         m_run = -INFINITY;
         l_run = 0.f;
       }
-      w_ok = mbar_wait(&s_full[X], t & 1, p.wait_ns);
+      const uint32_t s_col = C::S_COL + (t & 1) * 128;
+      const uint32_t o_col = C::O_COL + (cur_item & 1) * 128;
+      w_ok = mbar_wait(&s_full[t & 1], (t >> 1) & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
       // This warp's keys all belong to blocks the row's q-block does not list
@@ -870,11 +847,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(r[e]);
       }
       tmem_wait_ld();
-      if (C::SEP_P) {
-        // S_X(t) is in registers: the next QK may overwrite it
-        warp_arrive(&s_read[X]);
-        pv_pending = t > 0;
-      }
       float hmax = -INFINITY;
       if (!part_dead) {
         // masking: slots this row's q-block does not list, unused slots, keys >= N
@@ -903,15 +875,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         hmax = fmax3(fmax3(mx0, mx1, mx2), mx3, mx3);
       }
-      float tmax = hmax;
-      if (NH > 1) {
-        // agree on the row max with the other half (double-buffered by step
-        // parity); the barrier also orders both halves' S reads before any P write
-        float* xm = xmax + ((t & 1) * 4 + X * 2) * 128;
-        xm[h * 128 + row] = hmax;
-        if (!pair_sync()) { ok = false; break; }
-        tmax = fmaxf(hmax, xm[(h ^ 1) * 128 + row]);
-      }
+      // agree on the row max with the other half (double-buffered by step
+      // parity); the barrier also orders both halves' S reads before any P write
+      float* xm = xmax + (t & 1) * 2 * 128;
+      xm[h * 128 + row] = hmax;
+      if (!pair_sync()) { ok = false; break; }
+      const float tmax = fmaxf(hmax, xm[(h ^ 1) * 128 + row]);
       // lazy rescale (decided per warp: tcgen05.ld/st are warp-collective)
       const float m_new = fmaxf(m_run, tmax);
       const bool grow = m_run == -INFINITY ? (m_new > -INFINITY)
@@ -921,10 +890,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         alpha = (m_run == -INFINITY) ? 0.0f : fast_ex2((m_run - m_new) * c2);
         m_run = m_new;
       }
-      if (!wait_prev_pv(t)) { ok = false; break; }
       if (!first && __any_sync(0xffffffffu, grow)) {
-        // O_X holds PV up to the previous step, complete (see header); scale
-        // this warp's columns before any PV of this step
+        // O holds PV up to step t-2; wait for PV(t-1), then scale this warp's
+        // columns before the PV of this step
+        w_ok = mbar_wait(pv_done, (t - 1) & 1, p.wait_ns);
+        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll 1
         for (int c = 0; c < DW / 16; ++c) {
           uint32_t r[16];
@@ -967,76 +938,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             pk[c] = *reinterpret_cast<uint32_t*>(&hb);
           }
         }
-        // P (bf16 pairs): keys KW h + 32 q2 .. +31 -> columns KW/2 h + 16 q2
-        // (over S, or in the separate P columns)
-        tmem_st16(t_lane + p_col + h * (KW / 2) + q2 * 16, pk);
+        // P (bf16 pairs) over S: keys KW h + 32 q2 .. +31 -> columns KW/2 h + 16 q2
+        tmem_st16(t_lane + s_col + h * (KW / 2) + q2 * 16, pk);
       }
       float la0, la1, lb0, lb1;
       unpack2(ls2a, la0, la1);
       unpack2(ls2b, lb0, lb1);
       l_run = l_run * alpha + ((la0 + la1) + (lb0 + lb1));
       tmem_wait_st();
-      warp_arrive(&p_full[X]);
+      warp_arrive(&p_full[t & 1]);
+      if (pe && !epilogue()) { ok = false; break; }
       if (lastt) {
-        // ---- epilogue of the item: this warp's O columns
-        const int token = e_qt * 128 + row;
-        w_ok = mbar_wait(&o_done[X], items & 1, p.wait_ns);
-        if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-        tc_fence_after();
-        float l_tot = l_run;
-        if (NH > 1) {
-          float* xs = xsum + X * 2 * 128;
-          xs[h * 128 + row] = l_run;
-          if (!pair_sync()) { ok = false; break; }
-          l_tot = l_run + xs[(h ^ 1) * 128 + row];
-        }
-        const float inv_l = l_tot > 0.f ? 1.0f / l_tot : 0.f;
-        __nv_bfloat16* orow = p.o + ((long long)e_bh * p.N + token) * D + h * DW;
-#pragma unroll 1
-        for (int c = 0; c < DW / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32(t_lane + o_col + h * DW + c * 32, r);
-          tmem_wait_ld();
-          uint32_t packed[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * inv_l,
-                                                      __uint_as_float(r[2 * e + 1]) * inv_l);
-            packed[e] = *reinterpret_cast<uint32_t*>(&hb);
-          }
-          if (token < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
-                                  packed[4 * e + 3]);
-          }
-          if (RES && token < p.N) {
-            // the rounding residual of each element, so that O + residual
-            // carries the fp32 result to about 2^-16
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float a = __uint_as_float(r[2 * e]) * inv_l;
-              const float b = __uint_as_float(r[2 * e + 1]) * inv_l;
-              const float2 hi = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&packed[e]));
-              __nv_bfloat162 lo = __floats2bfloat162_rn(a - hi.x, b - hi.y);
-              packed[e] = *reinterpret_cast<uint32_t*>(&lo);
-            }
-            uint4* dr = reinterpret_cast<uint4*>(p.o_res + ((long long)e_bh * p.N + token) * D +
-                                                 h * DW + c * 32);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              dr[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2],
-                                 packed[4 * e + 3]);
-          }
-        }
-        warp_arrive(&o_free[X]);
-        if (h == 0 && p.lse != nullptr && token < p.N)
-          p.lse[(long long)e_bh * p.N + token] =
-              l_tot > 0.f ? (m_run * p.scale + logf(l_tot)) : -INFINITY;
-        ++items;
+        pe = true;
+        pe_item = cur_item;
+        pe_bh = e_bh;
+        pe_qt = e_qt;
+        pe_m = m_run;
+        pe_l = l_run;
       }
     }
+    if (ok && pe && !epilogue()) ok = false;
     if (!ok) {
       record_error(BSA_ERR_TIMEOUT);
       *(volatile int*)abort_flag = 1;

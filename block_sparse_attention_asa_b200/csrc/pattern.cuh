@@ -131,6 +131,17 @@ __device__ __forceinline__ int pattern_count(const PatternParams& p, int pattern
   return n;
 }
 
+// Row counts with the vertical stripe's taken once: its rows do not depend on
+// the q-block (every row keeps the stripe tokens of every frame).
+struct PatternCounter {
+  int stripe;
+  __device__ __forceinline__ explicit PatternCounter(const PatternParams& p)
+      : stripe(pattern_count(p, BSA_PATTERN_STRIPE, 0)) {}
+  __device__ __forceinline__ int operator()(const PatternParams& p, int pattern, int i) const {
+    return pattern == BSA_PATTERN_STRIPE ? stripe : pattern_count(p, pattern, i);
+  }
+};
+
 constexpr int kPatternScanThreads = 1024;
 constexpr int kPatternIds = BSA_PATTERN_TILE3D + 1;
 
@@ -147,6 +158,7 @@ __global__ void __launch_bounds__(kPatternScanThreads) pattern_rowptr_kernel(
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int h = blockIdx.x;
   if (tid < kPatternIds) s_tot[tid] = 0;
+  const PatternCounter count(p);
   __syncthreads();
   // totals of the patterns in use
   bool used[kPatternIds] = {};
@@ -154,7 +166,7 @@ __global__ void __launch_bounds__(kPatternScanThreads) pattern_rowptr_kernel(
   for (int pid = 0; pid < kPatternIds; ++pid) {
     if (!used[pid]) continue;
     long long part = 0;
-    for (int i = tid; i < p.nb; i += kPatternScanThreads) part += pattern_count(p, pid, i);
+    for (int i = tid; i < p.nb; i += kPatternScanThreads) part += count(p, pid, i);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
     if (lane == 0) atomicAdd(reinterpret_cast<unsigned long long*>(&s_tot[pid]),
@@ -177,7 +189,7 @@ __global__ void __launch_bounds__(kPatternScanThreads) pattern_rowptr_kernel(
   __syncthreads();
   for (int i0 = 0; i0 < p.nb; i0 += kPatternScanThreads) {
     const int i = i0 + tid;
-    const long long c = i < p.nb ? pattern_count(p, pid, i) : 0;
+    const long long c = i < p.nb ? count(p, pid, i) : 0;
     long long incl = c;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
