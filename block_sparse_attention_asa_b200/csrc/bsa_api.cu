@@ -594,7 +594,6 @@ int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
   p.col_idx = col_idx;
   p.capacity = col_capacity;
   cudaStream_t s = as_cuda(stream);
-  const long long units = (long long)H * p.nb;
   const long long rows = (long long)B * H * p.nb;
   bsa::pattern_rowptr_kernel<<<H, bsa::kPatternScanThreads, 0, s>>>(p);
   if (check_launch()) return BSA_ERR_CUDA;
@@ -607,7 +606,9 @@ int pattern_mask(const int32_t* head_pattern_host, int B, int H, int N, int blk,
     *nnz_out_host = nnz;
     if (nnz > col_capacity) return BSA_ERR_CAPACITY;
   }
-  bsa::pattern_write_kernel<<<ceil_div(units, 8), 256, 0, s>>>(p);
+  const dim3 wgrid(static_cast<unsigned>(ceil_div(p.nb, bsa::kPatternWriteWarps * bsa::kPatternRowsPerWarp)),
+                   static_cast<unsigned>(H));
+  bsa::pattern_write_kernel<<<wgrid, bsa::kPatternWriteWarps * 32, 0, s>>>(p);
   return check_launch();
 }
 

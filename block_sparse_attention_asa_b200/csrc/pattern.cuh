@@ -8,9 +8,10 @@
 // are runs of consecutive blocks in closed form from the token ranges.
 //
 // Two kernels: one CTA per head computes the rows' counts in closed form and
-// writes row_ptr (offsets from per-pattern totals and a block scan), then one
-// warp per row writes its runs of consecutive block ids (coalesced), once per
-// batch index (the pattern does not depend on b).  The output is write-bound.
+// writes row_ptr (offsets from per-pattern totals and a block scan), then each
+// warp writes a few rows of one head as runs of consecutive block ids
+// (coalesced), once per batch index (the pattern does not depend on b).  The
+// output is write-bound.
 #pragma once
 #include "common.cuh"
 
@@ -222,29 +223,66 @@ __global__ void __launch_bounds__(kPatternScanThreads) pattern_rowptr_kernel(
   if (h == 0 && tid == 0) p.row_ptr[0] = 0;
 }
 
-// One warp per row (h, i), every b: the runs, written as consecutive block
-// ids from the row's start (coalesced); nothing past the capacity is written.
-__global__ void __launch_bounds__(256) pattern_write_kernel(const __grid_constant__ PatternParams p) {
-  const int lane = threadIdx.x & 31;
-  const long long unit = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (unit >= (long long)p.H * p.nb) return;
-  const int h = static_cast<int>(unit / p.nb), i = static_cast<int>(unit % p.nb);
+// Rows of one head per CTA (kPatternRowsPerWarp consecutive rows per warp),
+// every b: each row's runs written as consecutive block ids from the row's
+// start, coalesced, 32-bit offsets from the row's start (nnz < 2^31).  The
+// rows of the full and vertical-stripe patterns do not depend on the q-block:
+// a full row is 0..nb-1 and the stripe row is built once per CTA in shared
+// memory (when it fits) and copied.  Nothing past the capacity is written.
+constexpr int kPatternRowsPerWarp = 4;
+constexpr int kPatternWriteWarps = 8;
+constexpr int kPatternRowSmem = 4096;   // stripe-row entries kept in shared memory
+__global__ void __launch_bounds__(kPatternWriteWarps * 32) pattern_write_kernel(
+    const __grid_constant__ PatternParams p) {
+  __shared__ int32_t s_row[kPatternRowSmem];
+  __shared__ int s_len;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int h = blockIdx.y;
   const int pattern = p.head_pattern[h];
-  for (int b = 0; b < p.B; ++b) {
-    const long long r = ((long long)b * p.H + h) * p.nb + i;
-    const long long start = p.row_ptr[r], end = p.row_ptr[r + 1];
-    long long pos = start;
-    pattern_runs(p, pattern, i, [&](int j0, int j1) {
-      const int n = j1 - j0 + 1;
-      for (int k = lane; k < n; k += 32) {
-        const long long at = pos + k;
-        if (at < end && at < p.capacity)
-          p.col_idx[at] = static_cast<int32_t>(j0 + k);
-        else if (at >= p.capacity && lane == 0)
-          record_error(BSA_ERR_CAPACITY);
+  const int i0 = (blockIdx.x * kPatternWriteWarps + warp) * kPatternRowsPerWarp;
+  bool from_smem = false;
+  int s_n = 0;
+  if (pattern == BSA_PATTERN_STRIPE) {   // uniform over the CTA
+    if (warp == 0) {
+      int pos = 0;
+      pattern_runs(p, pattern, 0, [&](int j0, int j1) {
+        const int n = j1 - j0 + 1;
+        for (int k = lane; k < n; k += 32)
+          if (pos + k < kPatternRowSmem) s_row[pos + k] = j0 + k;
+        pos += n;
+      });
+      if (lane == 0) s_len = pos;
+    }
+    __syncthreads();
+    s_n = s_len;
+    from_smem = s_n <= kPatternRowSmem;
+  }
+  for (int r = 0; r < kPatternRowsPerWarp; ++r) {
+    const int i = i0 + r;
+    if (i >= p.nb) break;
+    for (int b = 0; b < p.B; ++b) {
+      const long long row = ((long long)b * p.H + h) * p.nb + i;
+      const long long start = p.row_ptr[row], end = p.row_ptr[row + 1];
+      const long long lim = end < p.capacity ? end : p.capacity;
+      const int room = lim > start ? static_cast<int>(lim - start) : 0;   // entries it may write
+      if (lim < end && lane == 0) record_error(BSA_ERR_CAPACITY);
+      if (room == 0) continue;
+      int32_t* out = p.col_idx + start;
+      if (pattern == BSA_PATTERN_FULL) {
+        const int n = min(room, p.nb);
+        for (int k = lane; k < n; k += 32) out[k] = k;
+      } else if (from_smem) {
+        const int n = min(room, s_n);
+        for (int k = lane; k < n; k += 32) out[k] = s_row[k];
+      } else {
+        int pos = 0;
+        pattern_runs(p, pattern, i, [&](int j0, int j1) {
+          const int n = min(j1 - j0 + 1, room - pos);
+          for (int k = lane; k < n; k += 32) out[pos + k] = j0 + k;
+          pos += j1 - j0 + 1;
+        });
       }
-      pos += n;
-    });
+    }
   }
 }
 
