@@ -30,8 +30,11 @@
 //               into a K ring; the V boxes follow on a separate front, since V
 //               is needed one step later than K.  Q tiles go into two buffers,
 //               by item parity.
-//   warp 1      MMA issuer (one thread): S(t) = Q Kᵀ into S buffer t%2, then
-//               O += P(t-1) V for the previous step, with P read from TMEM.
+//   warp 1      MMA issuer (one thread): S(t) = Q Kᵀ into S buffer t%2 and
+//               O += P(t-1) V for the previous step (P read from TMEM), in
+//               whichever order their inputs arrive.  It and the producer
+//               poll with non-blocking barrier tests, so waiting on one
+//               barrier never delays their response to another.
 //   warp 2      allocates and releases TMEM.
 //   warps 4-11  softmax + epilogue.  Warp (q, h): rows 32q..32q+31 (TMEM lane
 //               quarter q), keys 64h..64h+63 of each 128-key step; the two
@@ -47,8 +50,8 @@
 //
 // TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [384,384+D).
 //
-// Issue order of the single MMA thread: QK(0), QK(1), PV(0), QK(2), PV(1), ...
-// i.e. in step t's slot: QK(t) into S(t%2), then PV(t-1).  Ordering facts:
+// The single MMA thread issues step t's pair, QK(t) into S(t%2) and PV(t-1),
+// in either order, and only after step t-1's pair.  Ordering facts:
 //   * tcgen05.mma ops issued by one thread execute in order.  QK(t) overwrites
 //     S(t%2) after PV(t-2) read P(t-2) from it (PV(t-2) was issued first, and
 //     waited for the softmax to finish step t-2);
@@ -329,7 +332,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int b = st.fills & 1;
       if (st.fills >= 2) {
         // one lane polls, the warp follows its answer
-        bool ready = lane == 0 && mbar_try_wait(&l_free[b], ((st.fills >> 1) - 1) & 1);
+        bool ready = lane == 0 && mbar_test_wait(&l_free[b], ((st.fills >> 1) - 1) & 1);
         if (!__shfl_sync(0xffffffffu, ready, 0)) return false;
       }
       int* h = hdr + b * 8;
@@ -463,7 +466,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // One pass of the V front: loads every V tile whose slot is free.
       auto v_front = [&]() -> bool {
         bool moved = false;
-        while (sv < sk && (sv < C::NV || mbar_try_wait(&v_free[sv % C::NV], ((sv / C::NV) - 1) & 1))) {
+        while (sv < sk && (sv < C::NV || mbar_test_wait(&v_free[sv % C::NV], ((sv / C::NV) - 1) & 1))) {
           const int* vqe = vq + (sv % C::VQ) * 12;
           const int vs = sv % C::NV;
           mbar_arrive_expect_tx(&v_full[vs], C::TILE);
@@ -517,9 +520,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // before.  While waiting, keep the V front going: that QK follows a
           // PV whose V tile this same thread's V front may still have to load.
           const int qb = P.qcount & 1;
-          if (P.qcount >= 2 && !mbar_try_wait(&q_free[qb], ((P.qcount >> 1) - 1) & 1)) {
+          if (P.qcount >= 2 && !mbar_test_wait(&q_free[qb], ((P.qcount >> 1) - 1) & 1)) {
             const uint64_t t0 = global_ns();
-            while (!mbar_try_wait(&q_free[qb], ((P.qcount >> 1) - 1) & 1)) {
+            while (!mbar_test_wait(&q_free[qb], ((P.qcount >> 1) - 1) & 1)) {
               v_front();
               if (global_ns() - t0 > p.wait_ns) return false;
             }
@@ -578,7 +581,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // queue entry it writes; entry sk reuses the step entry of sk - NM,
         // whose step's P was stored before QK(sk - NK) was issued)
         if (!P.flushed && sk - sv < C::VQ &&
-            (sk < C::NK || mbar_try_wait(&k_free[sk % C::NK], ((sk / C::NK) - 1) & 1))) {
+            (sk < C::NK || mbar_test_wait(&k_free[sk % C::NK], ((sk / C::NK) - 1) & 1))) {
           ok = k_step();
           if (!ok) break;
           if (used_ring) ++sk;
@@ -609,10 +612,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ================================================================ MMA issuer
-    // One thread issues every MMA of the CTA, in the order QK(t), PV(t-1):
-    // QK(t) needs only K(t) (and, on an item's first step, its Q tile), so the
-    // tensor pipe computes S(t) while the softmax works on step t-1; PV(t-1)
-    // waits until that step's P is stored.
+    // One thread issues every MMA of the CTA, step by step: QK(t) needs only
+    // K(t) (and, on an item's first step, its Q tile), so the tensor pipe
+    // computes S(t) while the softmax works on step t-1; PV(t-1) needs that
+    // step's P.  Whichever is ready first goes first.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
@@ -624,16 +627,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int pend = -1, pend_first = 0, pend_last = 0, pend_item = 0;
       int items = 0, cur_item = -1;
       bool ok = true, issued = false;
-      auto issue_pv = [&]() -> bool {
+      // PV of the pending step: its V tile, its P and (first step of an item)
+      // the O buffer, all polled without blocking
+      auto pv_ready = [&]() -> bool {
         const int sp = pend;
-        const int ob = pend_item & 1;
-        if (!mbar_wait(&v_full[sp % C::NV], (sp / C::NV) & 1, p.wait_ns)) return false;
+        if (!mbar_test_wait(&v_full[sp % C::NV], (sp / C::NV) & 1)) return false;
         // the first PV of an item overwrites its O buffer: the epilogue of
         // the item two before must have read it
         if (pend_first && pend_item >= 2 &&
-            !mbar_wait(&o_free[ob], ((pend_item >> 1) - 1) & 1, p.wait_ns))
+            !mbar_test_wait(&o_free[pend_item & 1], ((pend_item >> 1) - 1) & 1))
           return false;
-        if (!mbar_wait(&p_full[sp & 1], (sp >> 1) & 1, p.wait_ns)) return false;
+        return mbar_test_wait(&p_full[sp & 1], (sp >> 1) & 1);
+      };
+      auto issue_pv = [&]() {
+        const int sp = pend;
+        const int ob = pend_item & 1;
         tc_fence_after();
         const uint32_t t_o = tmem + C::O_COL + ob * 128;
         const uint32_t t_p = tmem + C::S_COL + (sp & 1) * 128;   // P over S
@@ -647,38 +655,60 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mma_commit(pv_done);
         if (pend_last) mma_commit(&o_done[ob]);
         pend = -1;
-        return true;
       };
+      // Step t's slot holds QK(t) and PV(t-1), issued in whichever order
+      // their inputs arrive (QK(t) needs PV(t-2) issued before it, which the
+      // previous slot guarantees; PV(t-1) needs QK(t-1), likewise).
       for (int t = 0; ok; ++t) {
         const int mi = t % C::NM;
-        if (!mbar_wait(&m_full[mi], (t / C::NM) & 1, p.wait_ns)) { ok = false; break; }
-        const int* sm = smeta + mi * C::SMETA_INTS;
-        if (sm[0] == kEntryEnd) {
-          if (pend >= 0 && !issue_pv()) ok = false;
-          break;
-        }
-        const int first = sm[1], lastt = sm[2], s = sm[22];
-        const int ks = s % C::NK;
-        if (!mbar_wait(&k_full[ks], (s / C::NK) & 1, p.wait_ns)) { ok = false; break; }
-        if (first) {
-          cur_item = items++;
-          if (!mbar_wait(&q_full[cur_item & 1], (cur_item >> 1) & 1, p.wait_ns)) { ok = false; break; }
-        }
-        tc_fence_after();
-        // S(t % 2) was last read as P(t-2) by PV(t-2), issued before this QK
-        const uint32_t t_s = tmem + C::S_COL + (t & 1) * 128;
-        const uint64_t dq = dq0 + static_cast<uint64_t>(((cur_item & 1) * C::TILE) >> 4);
-        const uint64_t dk = dk0 + static_cast<uint64_t>((ks * C::TILE) >> 4);
+        bool have = false, end = false, qk_done = false;
+        int first = 0, lastt = 0, s = 0;
+        uint64_t t0 = global_ns();
+        while (true) {
+          bool prog = false;
+          if (!have && mbar_test_wait(&m_full[mi], (t / C::NM) & 1)) {
+            const int* sm = smeta + mi * C::SMETA_INTS;
+            have = true;
+            end = sm[0] == kEntryEnd;
+            first = sm[1];
+            lastt = sm[2];
+            s = sm[22];
+            prog = true;
+          }
+          if (have && !end && !qk_done && mbar_test_wait(&k_full[s % C::NK], (s / C::NK) & 1) &&
+              (!first || mbar_test_wait(&q_full[items & 1], (items >> 1) & 1))) {
+            if (first) cur_item = items++;
+            tc_fence_after();
+            // S(t % 2) was last read as P(t-2) by PV(t-2), issued before this QK
+            const int ks = s % C::NK;
+            const uint32_t t_s = tmem + C::S_COL + (t & 1) * 128;
+            const uint64_t dq = dq0 + static_cast<uint64_t>(((cur_item & 1) * C::TILE) >> 4);
+            const uint64_t dk = dk0 + static_cast<uint64_t>((ks * C::TILE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
-          mma_ss(t_s, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
+              mma_ss(t_s, dq + off, dk + off, idesc_qk, kk > 0 ? 1u : 0u);
+            }
+            issued = true;
+            mma_commit(&k_free[ks]);
+            if (lastt) mma_commit(&q_free[cur_item & 1]);
+            mma_commit(&s_full[t & 1]);
+            qk_done = true;
+            prog = true;
+          }
+          if (pend >= 0 && pv_ready()) {
+            issue_pv();
+            prog = true;
+          }
+          if (pend < 0 && have && (end || qk_done)) break;
+          if (prog) {
+            t0 = global_ns();
+          } else if (global_ns() - t0 > p.wait_ns) {
+            ok = false;
+            break;
+          }
         }
-        issued = true;
-        mma_commit(&k_free[ks]);
-        if (lastt) mma_commit(&q_free[cur_item & 1]);
-        mma_commit(&s_full[t & 1]);
-        if (pend >= 0 && !issue_pv()) { ok = false; break; }
+        if (!ok || end) break;
         pend = s;
         pend_first = first;
         pend_last = lastt;
