@@ -297,9 +297,9 @@ class Layer:
                                dtype=torch.uint8, device=dev)
         self.o = torch.empty_like(self.q)
         self.lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-        # kernels per step: pool and select (ASA) or pattern count, scan and
+        # kernels per step: pool and select (ASA) or pattern row_ptr and
         # write; then the forward
-        self.launches = (2 if w.source == "asa" else 3) + 1
+        self.launches = 2 + 1
 
     def mask(self):
         w, b = self.w, self.bsa
@@ -547,6 +547,51 @@ def run_extra(bsa, args, head_layer: Layer, head_flops: float, pk: dict, local: 
     return ex
 
 
+def run_profile(args):
+    """One op of the workload run back to back (`--warmup` + `--steps` calls) with
+    nothing else around it, for a profiler's launch list or kernel capture:
+    `mask` (the layer's mask source), `forward` (on the layer's mask) or
+    `backward` (the training path: forward with the rounding residual once,
+    then the backward for a seeded dO).  Prints one line; not a benchmark."""
+    from block_sparse_attention_asa_b200 import bsa
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = workload(args.workload, args.keep, args.blk)
+    lay = Layer(bsa, w, dev)
+    lay.mask()
+    if args.profile == "mask":
+        call = lay.mask
+    elif args.profile == "forward":
+        call = lay.forward
+    else:
+        q, k, v = lay.q, lay.k, lay.v
+        B, H, N, d = q.shape
+        g = torch.Generator(device=dev).manual_seed(5)
+        dout = torch.randn(q.shape, generator=g, device=dev).to(torch.bfloat16)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(max(bsa.backward_workspace_size(B, H, N, d, w.blk), 4), dtype=torch.uint8,
+                         device=dev)
+        res = torch.empty_like(q)
+        bsa.bsa_forward_into(q, k, v, w.blk, lay.row_ptr, lay.col_idx, lay.o, lay.lse,
+                             workspace=lay.fws, o_residual=res)
+
+        def call():
+            bsa.bsa_backward_into(q, k, v, lay.o, dout, lay.lse, w.blk, lay.row_ptr, lay.col_idx,
+                                  dq, dk, dv, 0.0, ws, o_residual=res)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        call()
+    b.record()
+    torch.cuda.synchronize()
+    check_status(bsa, f"after {args.profile}")
+    print(json.dumps({"profile": args.profile, "workload": w.name, "calls": args.steps,
+                      "ms_per_call": a.elapsed_time(b) / args.steps}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -564,9 +609,14 @@ def main():
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other layers, the sweep and the backward (1 GPU only)")
     ap.add_argument("--extra-steps", type=int, default=5, help="timed steps of each extra layer")
+    ap.add_argument("--profile", choices=["mask", "forward", "backward"], default=None,
+                    help="run only this op of the workload back to back, for a profiler (1 GPU)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.profile is not None:
+        run_profile(args)
+        return
     rank, world, local = dist_setup(args.gpus)
     try:
         if args.impl == "reference":
