@@ -50,12 +50,12 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 
 
 # DRAM bytes (read + write) per bsa_fwd_kernel launch, from one ncu capture of
-# the bench's own command, keyed by workload and by the sha256 of the kernel
-# source the capture ran: once the kernel changes, the figure no longer applies
-# and the bench reports null.
+# this script's own `--profile forward` run on that workload, keyed by workload
+# and by the sha256 of the kernel source the capture ran: once the kernel
+# changes, the figure no longer applies and the bench reports null.
 FWD_TRAFFIC = {
-    ("wan2.1_1.3b_asa", "96289554c31f2322f6a5e5b32e686dc6dd3aafabd8be7fdf376cfb7edc0f9c88"):
-        309146368 + 85984768,
+    ("wan2.1_1.3b_asa", "4017ae624679036b3512ec6508f53ca5bf413e578eb5360d9a65f4c147c10ea7"):
+        303439872 + 84715264,
 }
 
 
