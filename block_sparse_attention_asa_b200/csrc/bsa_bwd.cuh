@@ -53,7 +53,7 @@ namespace bsa {
 
 // Element-wise warps: kBwdEltWarps / 4 per TMEM lane quarter, each taking a
 // contiguous part of the 128 columns of its rows.
-constexpr int kBwdEltWarps = 8;
+constexpr int kBwdEltWarps = 16;
 constexpr int kBwdParts = kBwdEltWarps / 4;
 constexpr int kBwdCols = 128 / kBwdParts;          // columns per element-wise warp
 constexpr int kBwdThreads = (4 + kBwdEltWarps) * 32;
@@ -190,23 +190,31 @@ __device__ __forceinline__ void zero_rows(__nv_bfloat16* g, long long bh, int t0
 template <int NC>
 __device__ __forceinline__ void store_acc_row(uint32_t taddr, float mul, __nv_bfloat16* dst,
                                               bool store) {
-  static_assert(NC % 32 == 0, "32-column loads");
+  static_assert(NC % 16 == 0, "16-column loads");
+  constexpr int EC = NC % 32 == 0 ? 32 : 16;   // columns per TMEM load
 #pragma unroll 1
-  for (int c = 0; c < NC / 32; ++c) {
+  for (int c = 0; c < NC / EC; ++c) {
     uint32_t r[32];
-    tmem_ld32(taddr + c * 32, r);
+    if constexpr (EC == 32) {
+      tmem_ld32(taddr + c * EC, r);
+    } else {
+      uint32_t r16[16];
+      tmem_ld16(taddr + c * EC, r16);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) r[e] = r16[e];
+    }
     tmem_wait_ld();
     uint32_t packed[16];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
+    for (int e = 0; e < EC / 2; ++e) {
       __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * mul,
                                                 __uint_as_float(r[2 * e + 1]) * mul);
       packed[e] = *reinterpret_cast<uint32_t*>(&hb);
     }
     if (store) {
-      uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+      uint4* d4 = reinterpret_cast<uint4*>(dst + c * EC);
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
+      for (int e = 0; e < EC / 8; ++e)
         d4[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
     }
   }
@@ -236,7 +244,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   int* meta = reinterpret_cast<int*>(smem + C::META_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   int* abort_flag = reinterpret_cast<int*>(smem + C::MISC_OFF + 4);
-  int* wcount = reinterpret_cast<int*>(smem + C::MISC_OFF + 16);    // [8]
+  int* wcount = reinterpret_cast<int*>(smem + C::MISC_OFF + 16);    // [warps]
   float* stage = reinterpret_cast<float*>(smem + C::STAGE_OFF);     // [2][LSE 128 | D 128]
   uint32_t* list = reinterpret_cast<uint32_t*>(smem + C::LIST_OFF);
 
