@@ -17,7 +17,9 @@
 //                        union of its q-blocks' rows, 128 keys per step as the
 //                        forward does: S = Q K^T and dP = dO V^T into TMEM,
 //                        dS (bf16) written over S, dQ += dS K with dS read
-//                        from TMEM.
+//                        from TMEM.  S is double-buffered (the kernel has one
+//                        accumulator, so the second one's columns are free):
+//                        S(s+1) runs during step s's element-wise pass.
 //   bsa_bwd_dkdv_kernel  item = (b.h, 128-key tile); walks the q-blocks whose
 //                        rows keep one of the tile's kv-blocks (binary search
 //                        in the ascending rows), 128 queries per step:
@@ -36,7 +38,8 @@
 // columns; one tile row per thread).
 //
 // TMEM columns: S [0,128), dP [128,256), first accumulator [256,256+D),
-// second accumulator [384,384+D).
+// second accumulator [384,384+D) (dK/dV kernel) or the odd steps' S (dQ
+// kernel).
 //
 // Ordering facts relied on (as in the forward): the tcgen05.mma ops of one
 // thread run in issue order, so the next step's S^T / dP^T may overwrite the
@@ -535,8 +538,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* res_full = bars;                     // resident Q, dO
   uint64_t* ring_full = res_full + 1;            // [NR] K, V of a step
   uint64_t* ring_free = ring_full + C::NR;       // [NR]
-  uint64_t* s_full = ring_free + C::NR;          // S, dP in TMEM
-  uint64_t* p_full = s_full + 1;                 // dS in TMEM (4 warps)
+  uint64_t* s_full = ring_free + C::NR;          // [2] S (by step parity) and dP in TMEM
+  uint64_t* p_full = s_full + 2;                 // dS in TMEM (element-wise warps)
   uint64_t* acc_done = p_full + 1;               // dQ complete
   uint64_t* drain = acc_done + 1;
   int* meta = reinterpret_cast<int*>(smem + C::META_OFF);
@@ -604,7 +607,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_free[s], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(p_full, kBwdEltWarps);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
@@ -682,40 +686,74 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t d_k = smem_desc(smem_u32(smem + C::RA_OFF), 16, 1024);           // K-major
       const uint64_t d_v = smem_desc(smem_u32(smem + C::RB_OFF), 16, 1024);           // K-major
       const uint64_t d_k_mn = smem_desc(smem_u32(smem + C::RA_OFF), C::CHUNK, 1024);  // MN-major
-      const uint32_t t_s = tmem + C::S_COL, t_dp = tmem + C::DP_COL, t_dq = tmem + C::ACC0_COL;
-      bool ok = mbar_wait(res_full, 0, p.wait_ns), issued = false;
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int slot = s % C::NR;
-        if (!mbar_wait(&ring_full[slot], (s / C::NR) & 1, p.wait_ns)) {
-          ok = false;
-          break;
-        }
+      // S is double-buffered (S of step s in the columns of parity s; the
+      // dQ kernel leaves the second accumulator's columns free), so S(s+1) =
+      // Q K(s+1)^T runs while the element-wise warps work on step s; dP has
+      // one buffer, so dP(s+1) follows the element-wise pass of step s.
+      const uint32_t t_dp = tmem + C::DP_COL, t_dq = tmem + C::ACC0_COL;
+      auto t_s = [&](int s) -> uint32_t { return tmem + ((s & 1) ? C::ACC1_COL : C::S_COL); };
+      auto issue_s = [&](int s) {
+        const uint64_t ro = static_cast<uint64_t>(((s % C::NR) * C::TILE) >> 4);
         tc_fence_after();
-        const uint64_t ro = static_cast<uint64_t>((slot * C::TILE) >> 4);
-        // S = Q K^T, dP = dO V^T (M = 128 queries, N = 128 keys, K = D)
+        // S = Q K^T (M = 128 queries, N = 128 keys, K = D)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
-          mma_ss(t_s, d_q + off, d_k + ro + off, idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(t_s(s), d_q + off, d_k + ro + off, idesc_s, kk > 0 ? 1u : 0u);
         }
+      };
+      auto issue_dp = [&](int s) {
+        const uint64_t ro = static_cast<uint64_t>(((s % C::NR) * C::TILE) >> 4);
+        // dP = dO V^T
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
           mma_ss(t_dp, d_do + off, d_v + ro + off, idesc_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full);
+        mma_commit(&s_full[s & 1]);   // S(s) and dP(s)
+      };
+      bool ok = mbar_wait(res_full, 0, p.wait_ns) && mbar_wait(&ring_full[0], 0, p.wait_ns);
+      bool issued = false;
+      if (ok) {
+        issue_s(0);
+        issue_dp(0);
         issued = true;
+      }
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int slot = s % C::NR;
+        const int s1 = s + 1, slot1 = s1 % C::NR;
+        // S(s+1) now if its K is already here (its buffer last held dS(s-1),
+        // read by dQ(s-1), issued before)
+        bool s1_done = false;
+        if (s1 < nsteps && mbar_test_wait(&ring_full[slot1], (s1 / C::NR) & 1)) {
+          issue_s(s1);
+          s1_done = true;
+        }
         if (!mbar_wait(p_full, s & 1, p.wait_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
         // dQ += dS K (M = 128 queries, N = D, K = 128 keys)
+        {
+          const uint64_t ro = static_cast<uint64_t>((slot * C::TILE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(t_dq, t_s + packed_col(kk * 16), d_k_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
-                 idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(t_dq, t_s(s) + packed_col(kk * 16),
+                   d_k_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4), idesc_acc,
+                   (s > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit(&ring_free[slot]);
+        if (s1 < nsteps) {
+          if (!s1_done) {
+            if (!mbar_wait(&ring_full[slot1], (s1 / C::NR) & 1, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            issue_s(s1);
+          }
+          issue_dp(s1);   // dP's buffer: the element-wise pass of step s has read dP(s)
+        }
       }
       if (ok) {
         mma_commit(acc_done);
@@ -769,13 +807,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (row_ok && sl < nvalid && ((me[9 + sl] >> qq) & 1)) live |= 1u << j;
         nk[j] = min(BLK, p.N - me[1 + sl] * BLK);
       }
-      w_ok = mbar_wait(s_full, s & 1, p.wait_ns);
+      w_ok = mbar_wait(&s_full[s & 1], (s >> 1) & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
+      const uint32_t s_col = (s & 1) ? C::ACC1_COL : C::S_COL;   // S of this step
 #pragma unroll
       for (int cc = 0; cc < kBwdCols / 32; ++cc) {
         uint32_t rs[32], rd[32];
-        tmem_ld32(t_lane + C::S_COL + cbase + cc * 32, rs);
+        tmem_ld32(t_lane + s_col + cbase + cc * 32, rs);
         tmem_ld32(t_lane + C::DP_COL + cbase + cc * 32, rd);
         tmem_wait_ld();
         uint32_t pd[16];
@@ -792,7 +831,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           pd[e] = *reinterpret_cast<uint32_t*>(&hd);
         }
         // dS (bf16 pairs) into the first half of this part's columns
-        tmem_st16(t_lane + C::S_COL + packed_col(cbase + cc * 32), pd);
+        tmem_st16(t_lane + s_col + packed_col(cbase + cc * 32), pd);
       }
       tmem_wait_st();
       warp_arrive(p_full);
