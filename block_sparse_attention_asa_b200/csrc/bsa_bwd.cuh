@@ -38,8 +38,9 @@
 // columns; one tile row per thread).
 //
 // TMEM columns: S [0,128), dP [128,256), first accumulator [256,256+D),
-// second accumulator [384,384+D) (dK/dV kernel) or the odd steps' S (dQ
-// kernel).
+// second accumulator [384,384+D) (dK/dV kernel at d = 128; at d = 64 it sits
+// at [320,384) and [384,512) holds the odd steps' S^T) or the odd steps' S
+// (dQ kernel).
 //
 // Ordering facts relied on (as in the forward): the tcgen05.mma ops of one
 // thread run in issue order, so the next step's S^T / dP^T may overwrite the
@@ -97,7 +98,7 @@ struct BwdCfg {
   static constexpr int RB_OFF = RA_OFF + NR * TILE;  // ring B (NR tiles)
   static constexpr int BAR_OFF = RB_OFF + NR * TILE;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int NBARS = 1 + 2 * NR + 5;
+  static constexpr int NBARS = 1 + 2 * NR + 6;
   static_assert(NBARS * 8 <= BAR_BYTES, "mbarriers must fit their area");
   static constexpr int META_OFF = BAR_OFF + BAR_BYTES;     // NR step entries
   static constexpr int META_INTS = 24;                     // [0] nvalid [1..8] ids [9..16] keep
@@ -232,6 +233,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         const __grid_constant__ CUtensorMap tm_do,   // box BLK rows
                         const BwdParams p) {
   using C = BwdCfg<D, BLK>;
+  // d = 64: dV [256, 320) and dK [320, 384) leave [384, 512) for a second S^T,
+  // so the next step's S^T runs during the element-wise pass; d = 128 has no
+  // room for it (the four regions take all 512 columns)
+  constexpr bool SDB = D == 64;
+  constexpr uint32_t DK_COL = SDB ? C::ACC0_COL + 64 : C::ACC1_COL;
+  auto s_col_of = [](int s) -> uint32_t { return (SDB && (s & 1)) ? 384u : C::S_COL; };
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -239,8 +246,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* res_full = bars;                     // resident K, V
   uint64_t* ring_full = res_full + 1;            // [NR] Q, dO of a step
   uint64_t* ring_free = ring_full + C::NR;       // [NR]
-  uint64_t* s_full = ring_free + C::NR;          // S^T, dP^T in TMEM
-  uint64_t* p_full = s_full + 1;                 // P^T, dS^T in TMEM (4 warps)
+  uint64_t* s_full = ring_free + C::NR;          // [2] S^T (by step parity), dP^T in TMEM
+  uint64_t* p_full = s_full + 2;                 // P^T, dS^T in TMEM (element-wise warps)
   uint64_t* acc_done = p_full + 1;               // dV, dK complete
   uint64_t* stage_bar = acc_done + 1;            // LSE/D staged (4 warps)
   uint64_t* drain = stage_bar + 1;
@@ -290,7 +297,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_free[s], 1);
     }
-    mbar_init(s_full, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     mbar_init(p_full, kBwdEltWarps);
     mbar_init(acc_done, 1);
     mbar_init(stage_bar, kBwdEltWarps);
@@ -371,45 +379,74 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t d_do = smem_desc(smem_u32(smem + C::RB_OFF), 16, 1024);         // K-major
       const uint64_t d_q_mn = smem_desc(smem_u32(smem + C::RA_OFF), C::CHUNK, 1024); // MN-major
       const uint64_t d_do_mn = smem_desc(smem_u32(smem + C::RB_OFF), C::CHUNK, 1024);
-      const uint32_t t_s = tmem + C::S_COL, t_dp = tmem + C::DP_COL;
-      const uint32_t t_dv = tmem + C::ACC0_COL, t_dk = tmem + C::ACC1_COL;
-      bool ok = mbar_wait(res_full, 0, p.wait_ns), issued = false;
-      for (int s = 0; ok && s < nsteps; ++s) {
-        const int slot = s % C::NR;
-        if (!mbar_wait(&ring_full[slot], (s / C::NR) & 1, p.wait_ns)) {
-          ok = false;
-          break;
-        }
+      const uint32_t t_dp = tmem + C::DP_COL;
+      const uint32_t t_dv = tmem + C::ACC0_COL, t_dk = tmem + DK_COL;
+      auto t_s = [&](int s) -> uint32_t { return tmem + s_col_of(s); };
+      auto issue_s = [&](int s) {
+        const uint64_t ro = static_cast<uint64_t>(((s % C::NR) * C::TILE) >> 4);
         tc_fence_after();
-        const uint64_t ro = static_cast<uint64_t>((slot * C::TILE) >> 4);
-        // S^T = K Q^T, dP^T = V dO^T (M = 128 keys, N = 128 queries, K = D)
+        // S^T = K Q^T (M = 128 keys, N = 128 queries, K = D)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
-          mma_ss(t_s, d_k + off, d_q + ro + off, idesc_s, kk > 0 ? 1u : 0u);
+          mma_ss(t_s(s), d_k + off, d_q + ro + off, idesc_s, kk > 0 ? 1u : 0u);
         }
+      };
+      auto issue_dp = [&](int s) {
+        const uint64_t ro = static_cast<uint64_t>(((s % C::NR) * C::TILE) >> 4);
+        // dP^T = V dO^T
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
           mma_ss(t_dp, d_v + off, d_do + ro + off, idesc_s, kk > 0 ? 1u : 0u);
         }
-        mma_commit(s_full);
+        mma_commit(&s_full[s & 1]);   // S^T(s) and dP^T(s)
+      };
+      bool ok = mbar_wait(res_full, 0, p.wait_ns) && mbar_wait(&ring_full[0], 0, p.wait_ns);
+      bool issued = false;
+      if (ok) {
+        issue_s(0);
+        issue_dp(0);
         issued = true;
+      }
+      for (int s = 0; ok && s < nsteps; ++s) {
+        const int slot = s % C::NR;
+        const int s1 = s + 1, slot1 = s1 % C::NR;
+        // double-buffered S^T (d = 64): S^T(s+1) now if its Q is already here
+        // (its buffer last held P^T(s-1), read by dV(s-1), issued before)
+        bool s1_done = false;
+        if (SDB && s1 < nsteps && mbar_test_wait(&ring_full[slot1], (s1 / C::NR) & 1)) {
+          issue_s(s1);
+          s1_done = true;
+        }
         if (!mbar_wait(p_full, s & 1, p.wait_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
         // dV += P^T dO, dK += dS^T Q (M = 128 keys, N = D, K = 128 queries)
+        {
+          const uint64_t ro = static_cast<uint64_t>((slot * C::TILE) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(t_dv, t_s + packed_col(kk * 16), d_do_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
-                 idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(t_dv, t_s(s) + packed_col(kk * 16), d_do_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
+                   idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(t_dk, t_dp + packed_col(kk * 16), d_q_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
-                 idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(t_dk, t_dp + packed_col(kk * 16), d_q_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
+                   idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
+        }
         mma_commit(&ring_free[slot]);
+        if (s1 < nsteps) {
+          if (!s1_done) {
+            if (!mbar_wait(&ring_full[slot1], (s1 / C::NR) & 1, p.wait_ns)) {
+              ok = false;
+              break;
+            }
+            issue_s(s1);   // single S^T buffer: after dV(s) read P^T(s)
+          }
+          issue_dp(s1);    // after dK(s) read dS^T(s), which lies over dP^T(s)
+        }
       }
       if (ok) {
         mma_commit(acc_done);
@@ -469,14 +506,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       warp_arrive(stage_bar);
       w_ok = mbar_wait(stage_bar, s & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-      w_ok = mbar_wait(s_full, s & 1, p.wait_ns);
+      w_ok = mbar_wait(&s_full[s & 1], (s >> 1) & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
       const float* stl = st + cbase;
+      const uint32_t s_col = s_col_of(s);   // S^T of this step
 #pragma unroll
       for (int cc = 0; cc < kBwdCols / 32; ++cc) {
         uint32_t rs[32], rd[32];
-        tmem_ld32(t_lane + C::S_COL + cbase + cc * 32, rs);
+        tmem_ld32(t_lane + s_col + cbase + cc * 32, rs);
         tmem_ld32(t_lane + C::DP_COL + cbase + cc * 32, rd);
         tmem_wait_ld();
         uint32_t pp[16], pd[16];
@@ -495,7 +533,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // bf16 pairs into the first half of this part's columns, over fp32
         // columns this warp has already read
-        tmem_st16(t_lane + C::S_COL + packed_col(cbase + cc * 32), pp);
+        tmem_st16(t_lane + s_col + packed_col(cbase + cc * 32), pp);
         tmem_st16(t_lane + C::DP_COL + packed_col(cbase + cc * 32), pd);
       }
       tmem_wait_st();
@@ -510,7 +548,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr int NC = D / kBwdParts;           // accumulator columns per part
       const long long row = ((long long)bh * p.N + key) * D + part * NC;
       store_acc_row<NC>(t_lane + C::ACC0_COL + part * NC, 1.0f, p.dv + row, key_ok);
-      store_acc_row<NC>(t_lane + C::ACC1_COL + part * NC, p.scale, p.dk + row, key_ok);
+      store_acc_row<NC>(t_lane + DK_COL + part * NC, p.scale, p.dk + row, key_ok);
     } else {
       record_error(BSA_ERR_TIMEOUT);
       *(volatile int*)abort_flag = 1;
