@@ -25,7 +25,10 @@
 //                        in the ascending rows), 128 queries per step:
 //                        S^T = K Q^T and dP^T = V dO^T into TMEM, P^T and dS^T
 //                        (bf16) written over them, dV += P^T dO and
-//                        dK += dS^T Q with P^T and dS^T read from TMEM.
+//                        dK += dS^T Q with P^T and dS^T read from TMEM; at
+//                        d = 64 in two halves of 64 queries, so that one
+//                        half's element-wise pass overlaps the other half's
+//                        MMAs.
 // Each tiled kernel keeps its own side's pair of tiles resident in shared
 // memory and streams the other side's gathered tiles through a two-deep ring.
 // No atomics: each gradient row is written once by the item that owns it, so
@@ -38,9 +41,8 @@
 // columns; one tile row per thread).
 //
 // TMEM columns: S [0,128), dP [128,256), first accumulator [256,256+D),
-// second accumulator [384,384+D) (dK/dV kernel at d = 128; at d = 64 it sits
-// at [320,384) and [384,512) holds the odd steps' S^T) or the odd steps' S
-// (dQ kernel).
+// second accumulator [384,384+D) (dK/dV kernel) or the odd steps' S (dQ
+// kernel).
 //
 // Ordering facts relied on (as in the forward): the tcgen05.mma ops of one
 // thread run in issue order, so the next step's S^T / dP^T may overwrite the
@@ -98,7 +100,7 @@ struct BwdCfg {
   static constexpr int RB_OFF = RA_OFF + NR * TILE;  // ring B (NR tiles)
   static constexpr int BAR_OFF = RB_OFF + NR * TILE;
   static constexpr int BAR_BYTES = 256;
-  static constexpr int NBARS = 1 + 2 * NR + 6;
+  static constexpr int NBARS = 1 + 2 * NR + 8;
   static_assert(NBARS * 8 <= BAR_BYTES, "mbarriers must fit their area");
   static constexpr int META_OFF = BAR_OFF + BAR_BYTES;     // NR step entries
   static constexpr int META_INTS = 24;                     // [0] nvalid [1..8] ids [9..16] keep
@@ -233,12 +235,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         const __grid_constant__ CUtensorMap tm_do,   // box BLK rows
                         const BwdParams p) {
   using C = BwdCfg<D, BLK>;
-  // d = 64: dV [256, 320) and dK [320, 384) leave [384, 512) for a second S^T,
-  // so the next step's S^T runs during the element-wise pass; d = 128 has no
-  // room for it (the four regions take all 512 columns)
-  constexpr bool SDB = D == 64;
-  constexpr uint32_t DK_COL = SDB ? C::ACC0_COL + 64 : C::ACC1_COL;
-  auto s_col_of = [](int s) -> uint32_t { return (SDB && (s & 1)) ? 384u : C::S_COL; };
+  // d = 64: each step's 128 queries are two halves of 64 (X = 0, 1): S^T_X and
+  // dP^T_X (N = 64 MMAs) into columns [64X, 64X + 64) of S^T and of dP^T,
+  // then dV += P^T_X dO_X and dK += dS^T_X Q_X (K = 64).  The element-wise
+  // warps of half X (the parts 2X and 2X + 1 of each lane quarter) depend only
+  // on half X's MMAs, so one half's element-wise pass runs while the tensor
+  // pipe works on the other half (measured on B200: CogVideoX backward 10.74
+  // -> 10.16 ms).  d = 128 keeps whole steps: there the half-rate N = 64 MMAs
+  // cost more than the overlap gains (Wan 3.62 -> 3.72 ms).
+  constexpr int NHALF = D == 64 ? 2 : 1;
+  constexpr int QH = 128 / NHALF;                // queries per half
+  constexpr int HW = kBwdEltWarps / NHALF;       // element-wise warps per half
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -246,11 +253,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* res_full = bars;                     // resident K, V
   uint64_t* ring_full = res_full + 1;            // [NR] Q, dO of a step
   uint64_t* ring_free = ring_full + C::NR;       // [NR]
-  uint64_t* s_full = ring_free + C::NR;          // [2] S^T (by step parity), dP^T in TMEM
-  uint64_t* p_full = s_full + 2;                 // P^T, dS^T in TMEM (element-wise warps)
-  uint64_t* acc_done = p_full + 1;               // dV, dK complete
-  uint64_t* stage_bar = acc_done + 1;            // LSE/D staged (4 warps)
-  uint64_t* drain = stage_bar + 1;
+  uint64_t* s_full = ring_free + C::NR;          // [2 halves] S^T_X, dP^T_X in TMEM
+  uint64_t* p_full = s_full + 2;                 // [2 halves] P^T_X, dS^T_X in TMEM
+  uint64_t* acc_done = p_full + 2;               // dV, dK complete
+  uint64_t* stage_bar = acc_done + 1;            // [2 halves] LSE/D of the half staged
+  uint64_t* drain = stage_bar + 2;
   int* meta = reinterpret_cast<int*>(smem + C::META_OFF);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   int* abort_flag = reinterpret_cast<int*>(smem + C::MISC_OFF + 4);
@@ -297,11 +304,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&ring_full[s], 1);
       mbar_init(&ring_free[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, kBwdEltWarps);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_full[x], HW);                 // the half's warps
+      mbar_init(&stage_bar[x], HW);
+    }
     mbar_init(acc_done, 1);
-    mbar_init(stage_bar, kBwdEltWarps);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -379,73 +387,69 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t d_do = smem_desc(smem_u32(smem + C::RB_OFF), 16, 1024);         // K-major
       const uint64_t d_q_mn = smem_desc(smem_u32(smem + C::RA_OFF), C::CHUNK, 1024); // MN-major
       const uint64_t d_do_mn = smem_desc(smem_u32(smem + C::RB_OFF), C::CHUNK, 1024);
-      const uint32_t t_dp = tmem + C::DP_COL;
-      const uint32_t t_dv = tmem + C::ACC0_COL, t_dk = tmem + DK_COL;
-      auto t_s = [&](int s) -> uint32_t { return tmem + s_col_of(s); };
-      auto issue_s = [&](int s) {
+      constexpr uint32_t idesc_h = idesc_bf16_f32(128, QH, 0, 0);   // N = the half's queries
+      const uint32_t t_s = tmem + C::S_COL, t_dp = tmem + C::DP_COL;
+      const uint32_t t_dv = tmem + C::ACC0_COL, t_dk = tmem + C::ACC1_COL;
+      // S^T_X = K Q_X^T and dP^T_X = V dO_X^T (M = 128 keys, N = 64 queries,
+      // K = D): Q_X, dO_X are rows 64X .. 64X+63 of the step's tiles
+      auto issue_sdp = [&](int s, int x) {
+        const uint64_t ro = static_cast<uint64_t>(((s % C::NR) * C::TILE + x * QH * 128) >> 4);
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
+          mma_ss(t_s + QH * x, d_k + off, d_q + ro + off, idesc_h, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
+          mma_ss(t_dp + QH * x, d_v + off, d_do + ro + off, idesc_h, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&s_full[x]);
+      };
+      // dV += P^T_X dO_X, dK += dS^T_X Q_X (M = 128 keys, N = D, K = 64 queries)
+      auto issue_acc = [&](int s, int x) {
         const uint64_t ro = static_cast<uint64_t>(((s % C::NR) * C::TILE) >> 4);
         tc_fence_after();
-        // S^T = K Q^T (M = 128 keys, N = 128 queries, K = D)
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
-          mma_ss(t_s(s), d_k + off, d_q + ro + off, idesc_s, kk > 0 ? 1u : 0u);
+        for (int k4 = 0; k4 < QH / 16; ++k4) {
+          const int kk = (QH / 16) * x + k4;          // 16-query group of the step
+          mma_ts(t_dv, t_s + packed_col(kk * 16), d_do_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
+                 idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
         }
-      };
-      auto issue_dp = [&](int s) {
-        const uint64_t ro = static_cast<uint64_t>(((s % C::NR) * C::TILE) >> 4);
-        // dP^T = V dO^T
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
-          mma_ss(t_dp, d_v + off, d_do + ro + off, idesc_s, kk > 0 ? 1u : 0u);
+        for (int k4 = 0; k4 < QH / 16; ++k4) {
+          const int kk = (QH / 16) * x + k4;
+          mma_ts(t_dk, t_dp + packed_col(kk * 16), d_q_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
+                 idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
         }
-        mma_commit(&s_full[s & 1]);   // S^T(s) and dP^T(s)
       };
       bool ok = mbar_wait(res_full, 0, p.wait_ns) && mbar_wait(&ring_full[0], 0, p.wait_ns);
       bool issued = false;
       if (ok) {
-        issue_s(0);
-        issue_dp(0);
+        for (int x = 0; x < NHALF; ++x) issue_sdp(0, x);
         issued = true;
       }
+      // order: ... acc_0(s), sdp_0(s+1), acc_1(s), sdp_1(s+1), ...  Each half's
+      // S^T/dP^T columns are rewritten only after that half's accumulating
+      // MMAs have been issued (same thread: they run in order).
       for (int s = 0; ok && s < nsteps; ++s) {
         const int slot = s % C::NR;
-        const int s1 = s + 1, slot1 = s1 % C::NR;
-        // double-buffered S^T (d = 64): S^T(s+1) now if its Q is already here
-        // (its buffer last held P^T(s-1), read by dV(s-1), issued before)
-        bool s1_done = false;
-        if (SDB && s1 < nsteps && mbar_test_wait(&ring_full[slot1], (s1 / C::NR) & 1)) {
-          issue_s(s1);
-          s1_done = true;
-        }
-        if (!mbar_wait(p_full, s & 1, p.wait_ns)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // dV += P^T dO, dK += dS^T Q (M = 128 keys, N = D, K = 128 queries)
-        {
-          const uint64_t ro = static_cast<uint64_t>((slot * C::TILE) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(t_dv, t_s(s) + packed_col(kk * 16), d_do_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
-                   idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(t_dk, t_dp + packed_col(kk * 16), d_q_mn + ro + static_cast<uint64_t>((kk * 2048) >> 4),
-                   idesc_acc, (s > 0 || kk > 0) ? 1u : 0u);
-        }
-        mma_commit(&ring_free[slot]);
-        if (s1 < nsteps) {
-          if (!s1_done) {
-            if (!mbar_wait(&ring_full[slot1], (s1 / C::NR) & 1, p.wait_ns)) {
+        const int s1 = s + 1;
+        for (int x = 0; x < NHALF; ++x) {
+          if (!mbar_wait(&p_full[x], s & 1, p.wait_ns)) {
+            ok = false;
+            break;
+          }
+          issue_acc(s, x);
+          if (x == NHALF - 1) mma_commit(&ring_free[slot]);   // the step's last reads of Q and dO
+          if (s1 < nsteps) {
+            if (x == 0 && !mbar_wait(&ring_full[s1 % C::NR], (s1 / C::NR) & 1, p.wait_ns)) {
               ok = false;
               break;
             }
-            issue_s(s1);   // single S^T buffer: after dV(s) read P^T(s)
+            issue_sdp(s1, x);
           }
-          issue_dp(s1);    // after dK(s) read dS^T(s), which lies over dP^T(s)
         }
       }
       if (ok) {
@@ -466,6 +470,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // [part * kBwdCols, part * kBwdCols + kBwdCols) of each step
     const int wq = warp & 3;
     const int part = (warp - 4) >> 2;
+    const int half = part / (4 / NHALF);         // query half of the step (d = 64: parts 2X, 2X+1)
     const int cbase = part * kBwdCols;
     const int sbase = cbase / BLK;                // first q slot of this part
     const int u = wq * 32 + lane;                 // key row of the tile
@@ -490,12 +495,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // stage LSE (log2 units) and D of the step's 128 queries; a query past N
       // or in an unused slot gets LSE = +inf (P = 0)
       float* st = stage + (s & 1) * 256;
-      if (gt < 128) {
-        const int sl = gt / BLK;
-        const int tok = me[1 + sl] * BLK + gt % BLK;
-        const bool valid = sl < nvalid && tok < p.N;
-        st[gt] = valid ? p.lse[(long long)bh * p.N + tok] * kLog2e : INFINITY;
-        st[128 + gt] = valid ? p.delta[(long long)bh * p.N + tok] : 0.f;
+      {
+        // the half's queries, staged by the half's first QH threads
+        const int ht = gt - half * HW * 32;
+        if (ht < QH) {
+          const int qi = half * QH + ht;          // query of the step
+          const int sl = qi / BLK;
+          const int tok = me[1 + sl] * BLK + qi % BLK;
+          const bool valid = sl < nvalid && tok < p.N;
+          st[qi] = valid ? p.lse[(long long)bh * p.N + tok] * kLog2e : INFINITY;
+          st[128 + qi] = valid ? p.delta[(long long)bh * p.N + tok] : 0.f;
+        }
       }
       uint32_t live = 0;   // q slots of the step whose q-block keeps this row's kv-block
 #pragma unroll
@@ -503,14 +513,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (sl < nvalid && ((me[9 + sl] >> kvb) & 1)) live |= 1u << sl;
       if (!key_ok) live = 0;
       const uint32_t live_p = live >> sbase;      // bit j: slot sbase + j
-      warp_arrive(stage_bar);
-      w_ok = mbar_wait(stage_bar, s & 1, p.wait_ns);
+      warp_arrive(&stage_bar[half]);
+      w_ok = mbar_wait(&stage_bar[half], s & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-      w_ok = mbar_wait(&s_full[s & 1], (s >> 1) & 1, p.wait_ns);
+      w_ok = mbar_wait(&s_full[half], s & 1, p.wait_ns);
       if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
       tc_fence_after();
       const float* stl = st + cbase;
-      const uint32_t s_col = s_col_of(s);   // S^T of this step
+      const uint32_t s_col = C::S_COL;
 #pragma unroll
       for (int cc = 0; cc < kBwdCols / 32; ++cc) {
         uint32_t rs[32], rd[32];
@@ -537,7 +547,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_st16(t_lane + C::DP_COL + packed_col(cbase + cc * 32), pd);
       }
       tmem_wait_st();
-      warp_arrive(p_full);
+      warp_arrive(&p_full[half]);
     }
     if (ok) {
       const bool w_ok = mbar_wait(acc_done, 0, p.wait_ns);
@@ -548,7 +558,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr int NC = D / kBwdParts;           // accumulator columns per part
       const long long row = ((long long)bh * p.N + key) * D + part * NC;
       store_acc_row<NC>(t_lane + C::ACC0_COL + part * NC, 1.0f, p.dv + row, key_ok);
-      store_acc_row<NC>(t_lane + DK_COL + part * NC, p.scale, p.dk + row, key_ok);
+      store_acc_row<NC>(t_lane + C::ACC1_COL + part * NC, p.scale, p.dk + row, key_ok);
     } else {
       record_error(BSA_ERR_TIMEOUT);
       *(volatile int*)abort_flag = 1;
